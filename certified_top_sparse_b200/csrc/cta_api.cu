@@ -1,0 +1,196 @@
+// C ABI of libcta: argument checks, launch planning, workspace layout and the
+// four-phase launch sequence of certified Top-k attention.  See include/cta.h
+// for the contract of every entry point.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "cta.h"
+#include "kernels.cuh"
+
+namespace cta {
+namespace {
+
+constexpr int kTargetCtas = 148 * 6;   // ~6 resident CTAs per SM over 148 SMs
+constexpr int64_t kMaxN = (int64_t)1 << 28;
+constexpr int kMaxChunks = 65535;      // grid.y limit
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+int ceil_log2(int64_t n) {
+  int l = 0;
+  while (((int64_t)1 << l) < n) ++l;
+  return l;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+  size_t u, cmax, sel, acc, part, status, total;
+};
+
+int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, double eps,
+              Plan* p) {
+  if (d != 64 && d != 128) return CTA_ERR_SHAPE;
+  if (n < 1 || n > kMaxN) return CTA_ERR_SHAPE;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return CTA_ERR_SHAPE;
+  if (batch < 1 || m < 1) return CTA_ERR_SHAPE;
+  const int64_t g = n_heads / n_kv_heads;
+  const int64_t gm = g * m;
+  const int64_t rows = (int64_t)batch * n_heads * m;
+  const int64_t groups = (int64_t)batch * n_kv_heads;
+  if (gm > (1 << 24) || rows > INT32_MAX || groups > 65535) return CTA_ERR_SHAPE;
+  memset(p, 0, sizeof(*p));
+  p->n = n;
+  p->rows = rows;
+  p->d = d;
+  p->gm = (int)gm;
+  p->groups = (int)groups;
+  p->rt_score = next_pow2((int)(gm < 8 ? gm : 8));
+  p->tiles_score = (int)((gm + p->rt_score - 1) / p->rt_score);
+  p->rt_out = next_pow2((int)(gm < 4 ? gm : 4));
+  p->tiles_out = (int)((gm + p->rt_out - 1) / p->rt_out);
+  // Chunk: enough CTAs to fill the GPU, a multiple of 256 keys, at most 4096
+  // keys (the logits of a tile are staged in shared memory).
+  const int64_t units = groups * p->tiles_score;
+  const int64_t want = (kTargetCtas + units - 1) / units;
+  int64_t chunk = (n + want - 1) / want;
+  chunk = ((chunk + 255) / 256) * 256;
+  if (chunk < 256) chunk = 256;
+  const int64_t max_chunk = (p->rt_score >= 8) ? 2048 : 4096;
+  if (chunk > max_chunk) chunk = max_chunk;
+  const int64_t nchunks = (n + chunk - 1) / chunk;
+  if (nchunks > kMaxChunks) return CTA_ERR_SHAPE;
+  p->chunk = (int)chunk;
+  p->nchunks = (int)nchunks;
+  p->scale = (float)(1.0 / sqrt((double)d));
+  int s = 62 - ceil_log2(n);
+  if (s > 52) s = 52;
+  p->mass_shift = s;
+  p->two_s = ldexpf(1.0f, s);
+  p->eps = eps;
+  return CTA_OK;
+}
+
+Layout layout(const Plan& p) {
+  Layout L;
+  size_t off = 0;
+  L.u = off;      off = align256(off + sizeof(float) * (size_t)p.rows * (size_t)p.n);
+  L.cmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks);
+  L.sel = off;    off = align256(off + sizeof(RowSel) * (size_t)p.rows);
+  L.acc = off;    off = align256(off + sizeof(double) * (size_t)p.rows * p.nchunks * 2 * p.d);
+  L.part = off;   off = align256(off + sizeof(Partial) * (size_t)p.rows * p.nchunks);
+  L.status = off; off = align256(off + sizeof(uint32_t));
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
+
+int record(void** ev, int i, cudaStream_t st) {
+  if (!ev) return CTA_OK;
+  return cudaEventRecord((cudaEvent_t)ev[i], st) == cudaSuccess ? CTA_OK : CTA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace cta
+
+using namespace cta;
+
+extern "C" {
+
+void cta_opts_init(cta_opts* o) {
+  if (!o) return;
+  memset(o, 0, sizeof(*o));
+  o->batch = 1;
+  o->m = 1;
+  o->dtype = CTA_BF16;
+}
+
+size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const cta_opts* o) {
+  cta_opts def;
+  cta_opts_init(&def);
+  if (!o) o = &def;
+  Plan p;
+  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, 0.5, &p) != CTA_OK) return 0;
+  return layout(p).total;
+}
+
+int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t n, int d,
+                            int n_heads, int n_kv_heads, double eps, void* out, int32_t* k_out,
+                            int32_t* idx_out, float* tv_out, const cta_opts* opts) {
+  if (!q || !K || !V || !out || !k_out || !idx_out || !tv_out) return CTA_ERR_ARG;
+  if (!(eps > 0.0 && eps < 1.0)) return CTA_ERR_ARG;
+  if (!opts) return CTA_ERR_WORKSPACE;  // the workspace is mandatory
+  if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return CTA_ERR_ARG;
+  Plan p;
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, eps, &p);
+  if (rc != CTA_OK) return rc;
+  p.want_err = opts->err_out != nullptr;
+  const Layout L = layout(p);
+  if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
+    return CTA_ERR_WORKSPACE;
+
+  char* ws = static_cast<char*>(opts->workspace);
+  float* u = reinterpret_cast<float*>(ws + L.u);
+  float* cmax = reinterpret_cast<float*>(ws + L.cmax);
+  RowSel* sel = reinterpret_cast<RowSel*>(ws + L.sel);
+  double* acc = reinterpret_cast<double*>(ws + L.acc);
+  Partial* part = reinterpret_cast<Partial*>(ws + L.part);
+  uint32_t* status = opts->status_dev ? opts->status_dev : reinterpret_cast<uint32_t*>(ws + L.status);
+  cudaStream_t st = static_cast<cudaStream_t>(opts->stream);
+  void** ev = opts->phase_events;
+
+  if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
+  if (launch_score(opts->dtype, q, K, u, cmax, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+  if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
+  if (launch_select(u, cmax, sel, k_out, tv_out, idx_out, p, status, st) != cudaSuccess)
+    return CTA_ERR_CUDA;
+  if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
+  if (launch_gather(opts->dtype, V, u, sel, acc, part, p, st) != cudaSuccess) return CTA_ERR_CUDA;
+  if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+  if (launch_finalize(opts->dtype, sel, acc, part, out, opts->err_out, opts->kl_out, p, status, st) !=
+      cudaSuccess)
+    return CTA_ERR_CUDA;
+  if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;
+  return CTA_OK;
+}
+
+int cta_dense_attn(const void* q, const void* K, const void* V, int64_t n, int d, int n_heads,
+                   int n_kv_heads, void* out, const cta_opts* opts) {
+  cta_opts def;
+  cta_opts_init(&def);
+  if (!opts) opts = &def;
+  if (!q || !K || !V || !out) return CTA_ERR_ARG;
+  if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V)) return CTA_ERR_ARG;
+  Plan p;
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, 0.5, &p);
+  if (rc != CTA_OK) return rc;
+  if (launch_dense(opts->dtype, q, K, V, out, n, d, p.rows, p.gm,
+                   static_cast<cudaStream_t>(opts->stream)) != cudaSuccess)
+    return CTA_ERR_CUDA;
+  return CTA_OK;
+}
+
+const char* cta_status_string(int status) {
+  switch (status) {
+    case CTA_OK: return "ok";
+    case CTA_ERR_ARG: return "invalid argument (NULL pointer, misaligned tensor, eps outside (0,1) or bad dtype)";
+    case CTA_ERR_SHAPE: return "unsupported shape (d not 64/128, n outside [1, 2^28], n_heads % n_kv_heads != 0)";
+    case CTA_ERR_WORKSPACE: return "workspace missing, not 256-byte aligned or smaller than cta_workspace_size()";
+    case CTA_ERR_CUDA: return "a CUDA launch or runtime call failed";
+    case CTA_ERR_NONFINITE: return "non-finite logit";
+    case CTA_ERR_TIMEOUT: return "timeout";
+    default: return "unknown status";
+  }
+}
+
+int cta_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,37 @@
+// Host-side launchers of the libcta kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "cta.h"
+#include "common.cuh"
+
+namespace cta {
+
+constexpr int kDtypeF32 = CTA_F32;
+constexpr int kDtypeBF16 = CTA_BF16;
+
+// Phase 1: logits u [rows, n] and per-(row, chunk) maxima cmax [rows, nchunks].
+cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, float* cmax,
+                         const Plan& p, uint32_t* status, cudaStream_t st);
+
+// Phase 2: per-row certified selection; writes sel, k_out, tv_out and idx_out.
+cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
+                          float* tv_out, int32_t* idx_out, const Plan& p, uint32_t* status,
+                          cudaStream_t st);
+
+// Phase 3: per-(tile, chunk) weighted value sums of kept (and dropped) keys.
+cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel,
+                          double* acc, Partial* part, const Plan& p, cudaStream_t st);
+
+// Phase 4: combine chunk partials into out, err, kl.
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const double* acc, const Partial* part,
+                            void* out, float* err_out, float* kl_out, const Plan& p,
+                            uint32_t* status, cudaStream_t st);
+
+// Dense reference attention (all keys, fp32 online softmax).
+cudaError_t launch_dense(int dtype, const void* q, const void* K, const void* V, void* out,
+                         int64_t n, int d, int64_t rows, int gm, cudaStream_t st);
+
+}  // namespace cta

@@ -1,0 +1,274 @@
+"""GPU <-> fp64 oracle parity of cta_certified_topk_attn, called through the C ABI.
+
+Small cases span several chunks with a ragged tail and run the oracle on
+every row; the five full-size workloads run the GPU in the launch
+configuration the benchmark times and compare sampled rows (whole
+(batch, KV-head) groups, which the oracle computes as problems of their own).
+Tolerances and exemption classes are stated in tests/parity.py.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from certified_top_sparse_b200 import workloads as W
+import certified_top_sparse_b200 as cta
+from parity import compare, group_rows, run_oracle, sub_problem, to_host
+
+pytestmark = pytest.mark.gpu
+
+REPORT = os.environ.get("CTA_PARITY_REPORT")
+
+
+def _report(name, rep):
+    if REPORT:
+        with open(REPORT, "a") as f:
+            f.write(json.dumps({"case": name, **rep}) + "\n")
+
+
+def gpu_run(prob: W.Problem, eps: float, q=None, **kw):
+    dev = torch.device("cuda")
+    qq = (prob.q if q is None else q).to(dev)
+    K, V = prob.K.to(dev), prob.V.to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = cta.cta_certified_topk_attn(qq, K, V, eps, status_dev=status, **kw)
+    torch.cuda.synchronize()
+    h = to_host(res)
+    h["status"] = int(status.item())
+    return h
+
+
+def check(prob, eps, name, **kw):
+    g = gpu_run(prob, eps, **kw)
+    assert g["status"] == 0, f"device status {g['status']:#x}"
+    o = run_oracle(prob, eps)
+    rep = compare(prob, eps, g, o)
+    _report(name, rep)
+    return g, o, rep
+
+
+# ---------------------------------------------------------------------------
+# small cases, every row checked
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 17, 255, 256, 257, 1000, 3001, 9999])
+def test_ragged_n_fp32_d64(n):
+    prob = W.tiny(n=n, d=64, n_heads=4)
+    check(prob, 0.01, f"tiny n={n}")
+
+
+def test_tiny_full_config():
+    prob = W.tiny()
+    g, o, rep = check(prob, prob.eps, "tiny (full config)")
+    assert rep["exact"] == prob.rows
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.float32, 128),
+                                     (torch.bfloat16, 64), (torch.bfloat16, 128)])
+@pytest.mark.parametrize("eps", [0.3, 0.01, 1e-4])
+def test_dtype_and_head_dim(dtype, d, eps):
+    prob = W.decode32k(batch=2, n_heads=8, n_kv_heads=2, n=5000 + d, d=d)
+    if dtype == torch.float32:
+        prob.q, prob.K, prob.V = prob.q.float(), prob.K.float(), prob.V.float()
+    check(prob, eps, f"decode {dtype} d={d} eps={eps}")
+
+
+@pytest.mark.parametrize("n_heads,n_kv,m", [(8, 8, 1), (16, 2, 1), (6, 2, 3), (4, 1, 5), (2, 2, 33)])
+def test_gqa_groups_and_query_rows(n_heads, n_kv, m):
+    rng = np.random.default_rng(n_heads * 100 + m)
+    d, n = 64, 2500
+    q = torch.from_numpy(rng.standard_normal((2, n_heads, m, d)).astype(np.float32) * 1.5)
+    K = torch.from_numpy(rng.standard_normal((2, n_kv, n, d)).astype(np.float32))
+    V = torch.from_numpy(rng.standard_normal((2, n_kv, n, d)).astype(np.float32))
+    prob = W.Problem("gqa", q, K, V, 0.05, 2, n_heads, n_kv, m, n, d)
+    check(prob, 0.05, f"gqa h={n_heads} kv={n_kv} m={m}")
+
+
+def test_bert_small_all_query():
+    prob = W.bert(batch=1, n_heads=4, n=512, d=64, sharp_from=2)
+    g, o, rep = check(prob, prob.eps, "bert small")
+
+
+def test_sweep_cell_small():
+    prob = W.sweep_cell(n=4096, sigma=2.0, m=64)
+    for eps in W.SWEEP_EPS:
+        check(prob, eps, f"sweep n=4096 eps={eps}")
+
+
+# ---------------------------------------------------------------------------
+# degenerate inputs: ties, radix narrowing, extremes
+
+
+def test_uniform_logits_all_ties_radix_path():
+    """q = 0: every logit ties, the boundary bin holds all n keys (> shared
+    capacity) and the radix narrowing over the key index decides the cut:
+    k = least k with (n-k)/n <= eps, kept keys 0..k-1."""
+    n, d = 100003, 64
+    rng = np.random.default_rng(5)
+    q = torch.zeros(1, 2, 1, d)
+    K = torch.from_numpy(rng.standard_normal((1, 2, n, d)).astype(np.float32))
+    V = torch.from_numpy(rng.standard_normal((1, 2, n, d)).astype(np.float32))
+    prob = W.Problem("uniform", q, K, V, 0.3, 1, 2, 2, 1, n, d)
+    g, o, rep = check(prob, 0.3, "uniform ties n=100003")
+    assert np.all(g["k"] == o["k"])
+    assert g["idx"][0, : g["k"][0]].tolist() == list(range(g["k"][0]))
+
+
+def test_near_uniform_logits_radix_on_logit_bits():
+    """Logits spread over ~1e-4: all keys share the first value bin, so the
+    cut is found by radix digits of the logit bits."""
+    n, d = 60000, 64
+    prob = W.tiny(n=n, d=d, n_heads=2, sigmas=(1e-4, 3e-4))
+    check(prob, 0.2, "near-uniform n=60000")
+
+
+def test_one_dominant_key():
+    n, d = 20000, 64
+    q = torch.zeros(1, 1, 1, d)
+    q[..., 0] = 8.0
+    K = torch.zeros(1, 1, n, d)
+    K[0, 0, 777, 0] = 40.0
+    V = torch.randn(1, 1, n, d, generator=torch.Generator().manual_seed(3))
+    prob = W.Problem("spike", q, K, V, 1e-3, 1, 1, 1, 1, n, d)
+    g, o, rep = check(prob, 1e-3, "one dominant key")
+    assert g["k"][0] == 1 and g["idx"][0, 0] == 777
+
+
+@pytest.mark.parametrize("eps", [0.999, 0.5, 1e-7])
+def test_extreme_eps(eps):
+    prob = W.tiny(n=4096, d=64, n_heads=3)
+    check(prob, eps, f"extreme eps={eps}")
+
+
+def test_no_err_path_matches_err_path_bitwise():
+    prob = W.decode32k(batch=1, n_heads=8, n_kv_heads=2, n=7000, d=128)
+    a = gpu_run(prob, 0.1)
+    b = gpu_run(prob, 0.1, want_err=False, want_kl=False)
+    for key in ("k", "tv"):
+        assert np.array_equal(a[key], b[key])
+    for r in range(prob.rows):
+        assert np.array_equal(a["idx"][r, : a["k"][r]], b["idx"][r, : b["k"][r]])
+    assert np.array_equal(a["out"], b["out"])
+
+
+def test_deterministic_repeat():
+    prob = W.decode32k(batch=1, n_heads=8, n_kv_heads=2, n=20000, d=128)
+    a = gpu_run(prob, 0.01)
+    b = gpu_run(prob, 0.01)
+    for key in ("k", "tv", "err", "kl", "out"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_nonfinite_input_sets_status():
+    prob = W.tiny(n=3000, d=64, n_heads=2)
+    prob.K[0, 1, 1234, 5] = float("nan")
+    g = gpu_run(prob, 0.01)
+    assert g["status"] & cta.CTA_DEV_NONFINITE
+    # the row that does not read the bad key is unaffected
+    o = run_oracle(W.Problem("row0", prob.q[:, :1].contiguous(), prob.K[:, :1].contiguous(),
+                             prob.V[:, :1].contiguous(), 0.01, 1, 1, 1, 1, prob.n, prob.d), 0.01)
+    assert g["k"][0] == o["k"][0]
+
+
+def test_dense_reference_matches_oracle():
+    import oracle
+    for prob in (W.tiny(n=3333, d=64, n_heads=4),
+                 W.decode32k(batch=1, n_heads=8, n_kv_heads=2, n=4444, d=128)):
+        dev = torch.device("cuda")
+        out = cta.cta_dense_attn(prob.q.to(dev), prob.K.to(dev), prob.V.to(dev))
+        torch.cuda.synchronize()
+        og = out.float().reshape(prob.rows, -1).cpu().numpy()
+        oo = oracle.dense_attn(W.raw_words(prob.q), W.raw_words(prob.K), W.raw_words(prob.V),
+                               n_heads=prob.n_heads, n_kv_heads=prob.n_kv_heads,
+                               dtype=oracle.F32 if prob.q.dtype == torch.float32 else oracle.BF16)
+        tol = 1e-5 if prob.q.dtype == torch.float32 else 3e-3
+        scale = np.abs(oo).max(axis=1, keepdims=True)
+        assert np.all(np.abs(og - oo) <= tol * scale)
+
+
+def test_err_equals_distance_to_dense_fp32():
+    """GPU-internal identity: err = ||Attn - Attn_k|| with Attn from cta_dense_attn."""
+    prob = W.tiny(n=8192, d=64, n_heads=6)
+    dev = torch.device("cuda")
+    q, K, V = prob.q.to(dev), prob.K.to(dev), prob.V.to(dev)
+    res = cta.cta_certified_topk_attn(q, K, V, 0.01)
+    dense = cta.cta_dense_attn(q, K, V)
+    torch.cuda.synchronize()
+    direct = (dense - res["out"]).double().reshape(prob.rows, -1).norm(dim=1).cpu().numpy()
+    err = res["err"].double().reshape(-1).cpu().numpy()
+    assert np.allclose(err, direct, rtol=1e-3, atol=1e-6)
+    # TV = 1 - exp(-KL) between the two independent reductions
+    tv = res["tv"].double().reshape(-1).cpu().numpy()
+    kl = res["kl"].double().reshape(-1).cpu().numpy()
+    assert np.all(np.abs(tv + np.expm1(-kl)) <= 1e-6)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads: GPU at full size, oracle on sampled groups
+
+
+def _sampled(prob, eps, groups, name, q=None):
+    g = gpu_run(prob, eps, q=q)
+    assert g["status"] == 0
+    reps = []
+    for (b, kvh) in groups:
+        sub = sub_problem(prob, b, kvh, q=q)
+        o = run_oracle(sub, eps)
+        reps.append(compare(sub, eps, g, o, rows=group_rows(prob, b, kvh)))
+    rep = {"rows": sum(r["rows"] for r in reps), "exact": sum(r["exact"] for r in reps),
+           "differing_exempt": sum(r["differing_exempt"] for r in reps),
+           "classM": {w: sum(r["classM"][w] for r in reps) for w in reps[0]["classM"]},
+           "classT": sum(r["classT"] for r in reps),
+           "max_out_rel": max(r["max_out_rel"] for r in reps)}
+    _report(name, rep)
+    return g
+
+
+def test_full_decode32k_sampled():
+    prob = W.decode32k()
+    _sampled(prob, prob.eps, [(0, 0), (1, 5), (3, 7)], "decode32k full (3 sampled groups)")
+
+
+@pytest.mark.parametrize("eps", [0.01, 0.1])
+def test_full_decode128k_sampled(eps):
+    prob = W.decode128k(steps=3)
+    for t in range(3):
+        _sampled(prob, eps, [(0, t), (0, 7 - t)], f"decode128k eps={eps} step={t}",
+                 q=prob.meta["q_steps"][t])
+
+
+def test_full_bert_sampled():
+    prob = W.bert()
+    g = gpu_run(prob, prob.eps)
+    assert g["status"] == 0
+    for (b, h) in [(0, 0), (3, 5), (5, 6), (7, 11)]:
+        sub = W.Problem("bert", prob.q[b:b + 1, h:h + 1].contiguous(),
+                        prob.K[b:b + 1, h:h + 1].contiguous(), prob.V[b:b + 1, h:h + 1].contiguous(),
+                        prob.eps, 1, 1, 1, prob.m, prob.n, prob.d)
+        o = run_oracle(sub, prob.eps)
+        rep = compare(sub, prob.eps, g, o, rows=group_rows(prob, b, h))
+        _report(f"bert full (b={b}, h={h})", rep)
+
+
+def test_full_sweep_gaussian_rule_and_sampled_parity():
+    from scipy import special
+    for n in W.SWEEP_N:
+        for sigma in W.SWEEP_SIGMA:
+            prob = W.sweep_cell(n=n, sigma=sigma)
+            for eps in W.SWEEP_EPS:
+                g = gpu_run(prob, eps)
+                assert g["status"] == 0
+                frac = g["k"].mean() / n
+                pred = float(special.ndtr(-(sigma + special.ndtri(eps))))
+                if n >= 65536:
+                    assert abs(frac - pred) <= 0.01, (n, sigma, eps, frac, pred)
+                rows = np.arange(0, prob.m, 37)
+                sub = W.Problem("sweep", prob.q[:, :, rows].contiguous(), prob.K, prob.V, eps, 1,
+                                1, 1, len(rows), n, prob.d)
+                o = run_oracle(sub, eps)
+                rep = compare(sub, eps, g, o, rows=rows)
+                rep["k_over_n"] = frac
+                rep["rule"] = pred
+                _report(f"sweep n={n} sigma={sigma} eps={eps}", rep)
