@@ -1,0 +1,427 @@
+"""Benchmark of certified Top-k attention (libcta) on B200.
+
+Headline workload: 128K GQA decode - batch 1, 32 query heads, 8 KV heads,
+d = 128, n = 131072 bf16 KV cache with sink / recent-window / needle
+structure, eps = 0.01, a fresh query set every step (64-step cycle).  One
+step = one call of cta_certified_topk_attn over all 32 query heads (logits,
+certified selection, head/tail value sums, finalisation, err and KL on).
+The metric is query heads per second; the roofline is HBM bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libcta|reference]
+
+N > 1 runs under torchrun, one process per GPU, each rank an independent
+replica of the workload (rows shard with no exchange step: weak scaling); the
+time is the maximum over ranks.  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "certified top-k attn query-heads/s & HBM GB/s (% of peak) at n=32K/128K"
+UNIT = "query-heads/s"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ("score.cu", "select.cu", "gather.cu", "common.cuh")
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (tested on CPU with gloo)
+
+
+def dist_env():
+    """(rank, world, local_rank) from torchrun's environment, or (0, 1, 0)."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Largest value of x over all ranks (the job's time is its slowest rank)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(rows_per_step: int, steps: int, world: int, seconds: float) -> float:
+    """Whole-job throughput: the units every rank processed / the slowest time."""
+    return rows_per_step * steps * world / seconds
+
+
+# --------------------------------------------------------------------------
+# measurement helpers
+
+
+def measured_peaks() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "certified_top_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when it is missing or the kernel sources changed since the capture."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = f"/tmp/cta_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self) -> dict:
+        try:
+            lines = [l.split(",") for l in open(self.path).read().strip().splitlines()]
+        except Exception:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = [[c.strip() for c in l] for l in lines if len(l) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [s for s in sm if mx and s >= 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# the libcta arm
+
+
+def algorithmic_bytes(prob, k_rows=None) -> dict:
+    """Bytes one step must move at minimum: K once per KV head for the logits,
+    every V row once per KV head for the output (the exact head-tail error
+    needs the dropped rows too), q and outputs (negligible), and the kept
+    indices written (reported separately)."""
+    kv = prob.batch * prob.n_kv_heads * prob.n * prob.d * prob.K.element_size()
+    idx = 0 if k_rows is None else int(k_rows.sum()) * 4
+    return {"score": kv, "gather": kv, "step": 2 * kv, "idx_write": idx}
+
+
+def run_libcta(args, rank, world, local_rank) -> dict | None:
+    import torch
+    import certified_top_sparse_b200 as cta
+    from certified_top_sparse_b200 import workloads as W
+
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    prob = W.decode128k() if args.workload == "decode128k" else W.decode32k()
+    eps = args.eps if args.eps is not None else prob.eps
+    if args.workload == "decode128k":
+        q_steps = prob.meta["q_steps"].to(device)                   # [64, B, H, 1, d]
+    else:
+        q_steps = prob.q.unsqueeze(0).to(device)
+    K, V = prob.K.to(device), prob.V.to(device)
+    rows = prob.rows
+    rshape = (prob.batch, prob.n_heads, prob.m)
+    out = torch.empty_like(q_steps[0])
+    k_out = torch.empty(rshape, dtype=torch.int32, device=device)
+    idx = torch.empty((*rshape, prob.n), dtype=torch.int32, device=device)
+    tv = torch.empty(rshape, dtype=torch.float32, device=device)
+    err = torch.empty(rshape, dtype=torch.float32, device=device)
+    kl = torch.empty(rshape, dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                            batch=prob.batch), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    nq = q_steps.shape[0]
+
+    def step(t, events=None):
+        cta.cta_certified_topk_attn(q_steps[t % nq], K, V, eps, out=out, k_out=k_out, idx_out=idx,
+                                    tv_out=tv, err_out=err, kl_out=kl, workspace=ws,
+                                    status_dev=status, stream=stream, phase_events=events)
+
+    for t in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize(device)
+    assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
+
+    # per-phase events, one set per step, recorded inside the timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for s in ev:
+        for e in s:
+            e.record(stream)
+    handles = [(ctypes.c_void_p * 5)(*[e.cuda_event for e in s]) for s in ev]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(device)
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_id = visible.split(",")[local_rank].strip() if visible else str(local_rank)
+    with ClockSampler(gpu_id) as clocks:
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        start.record(stream)
+        for t in range(args.steps):
+            step(t, ctypes.cast(handles[t], ctypes.c_void_p))
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+    ms = start.elapsed_time(stop)
+    phase = [0.0] * 4
+    for s in ev:
+        for j in range(4):
+            phase[j] += s[j].elapsed_time(s[j + 1])
+    phase = [p / args.steps for p in phase]
+    seconds = max_over_ranks(ms / 1e3, dist, device)
+    value = aggregate(rows, args.steps, world, seconds)
+
+    # end to end through the public call with host buffers: q in, results out
+    host_q = q_steps.cpu().pin_memory()
+    host_out = torch.empty_like(out, device="cpu").pin_memory()
+    host_small = torch.empty((4, *rshape), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 2000))
+    q_dev = torch.empty_like(q_steps[0])
+
+    def e2e_step(t):
+        q_dev.copy_(host_q[t % nq], non_blocking=True)
+        cta.cta_certified_topk_attn(q_dev, K, V, eps, out=out, k_out=k_out, idx_out=idx, tv_out=tv,
+                                    err_out=err, kl_out=kl, workspace=ws, status_dev=status,
+                                    stream=stream)
+        host_out.copy_(out, non_blocking=True)
+        host_small[0].copy_(k_out.view(torch.float32), non_blocking=True)  # raw int32 bits
+        host_small[1].copy_(tv, non_blocking=True)
+        host_small[2].copy_(err, non_blocking=True)
+        host_small[3].copy_(kl, non_blocking=True)
+
+    for t in range(3):
+        e2e_step(t)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for t in range(e2e_steps):
+        e2e_step(t)
+    e2.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_seconds = max_over_ranks(s2.elapsed_time(e2) / 1e3, dist, device)
+    h2d = q_steps[0].numel() * q_steps[0].element_size()
+    d2h = out.numel() * out.element_size() + 4 * rows * 4
+
+    assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
+    nbytes = algorithmic_bytes(prob, k_out.reshape(-1).cpu())
+    peak, peak_kind = measured_peaks()
+    names = ("score", "select", "gather", "finalize")
+    dom = max(range(4), key=lambda j: phase[j])
+    dom_name = names[dom]
+    dom_bytes = nbytes.get(dom_name, 0)
+    achieved = dom_bytes / (phase[dom] / 1e3) / 1e9 if dom_bytes else None
+    step_gbs = nbytes["step"] / (seconds / args.steps) / 1e9
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": seconds * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": (f"{args.workload}: batch {prob.batch}, {prob.n_heads} query heads, "
+                         f"{prob.n_kv_heads} KV heads, d={prob.d}, n={prob.n}, bf16 KV cache "
+                         f"(sink/window/needle structure), eps={eps}, "
+                         + ("fresh queries each step (64-step cycle)" if nq > 1 else "fixed queries")),
+            "input_dtype": "bf16", "query_heads_per_step": rows, "err_and_kl": True,
+            "l2": "inputs larger than L2 (K+V %.0f MB per step); no flush" % (nbytes["step"] / 1e6),
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak if achieved else None, "traffic": profiled_traffic(dom_name),
+            "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_kind,
+        },
+        "step_roofline": {"achieved_gbs": step_gbs, "frac": step_gbs / peak,
+                          "algorithmic_bytes_per_step": nbytes["step"],
+                          "idx_write_bytes_per_step": nbytes["idx_write"]},
+        "phase_ms": dict(zip(names, [round(p, 5) for p in phase])),
+        "e2e": {"value": aggregate(rows, e2e_steps, world, e2e_seconds), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "q copied in from pinned host memory, out/k/tv/err/kl copied back every "
+                        "step; the KV cache is resident and idx stays on the device"},
+        "gpu_launches": 4 * args.steps,
+        "k_over_n_mean": float(k_out.float().mean().item() / prob.n),
+        "clocks": clocks.summary(),
+    }
+    if dist is not None:
+        dist.destroy_process_group()
+    return res if rank == 0 else None
+
+
+# --------------------------------------------------------------------------
+# the oracle (CPU) as the reference arm and the cpu_baseline leg
+
+
+def oracle_sample(prob, q, n_keys: int, rows: int, threads: int):
+    """Run the oracle on the first `rows` query heads of one step over the
+    first `n_keys` keys; returns wall seconds."""
+    import oracle
+    from certified_top_sparse_b200 import workloads as W
+    g = prob.n_heads // prob.n_kv_heads
+    kv_groups = max(1, math.ceil(rows / g))
+    qs = q[:, : kv_groups * g].contiguous()
+    K = prob.K[:, :kv_groups, :n_keys].contiguous()
+    V = prob.V[:, :kv_groups, :n_keys].contiguous()
+    t0 = time.perf_counter()
+    oracle.certified_topk_attn(W.raw_words(qs), W.raw_words(K), W.raw_words(V), prob.eps,
+                               n_heads=kv_groups * g, n_kv_heads=kv_groups, dtype=oracle.BF16,
+                               batch=prob.batch, threads=threads)
+    return time.perf_counter() - t0, kv_groups * g * prob.batch
+
+
+def cpu_baseline(prob, budget_rows: int | None = None) -> dict:
+    """The oracle as it stands, all host cores, on whole rows of one step."""
+    threads = os.cpu_count() or 1
+    q = prob.meta["q_steps"][1] if "q_steps" in prob.meta else prob.q
+    rows = budget_rows or min(prob.n_heads * prob.batch, max(prob.n_heads // prob.n_kv_heads,
+                                                              threads))
+    secs, done = oracle_sample(prob, q, prob.n, rows, threads)
+    return {"value": done / secs, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} query heads of one decode step at full n={prob.n} "
+                      f"({secs:.2f} s wall on {threads} threads)"}
+
+
+def run_reference(args, rank, world) -> dict | None:
+    """bench.py --impl reference: the fp64 oracle on host cores, rank 0 only."""
+    if rank != 0:
+        return None
+    from certified_top_sparse_b200 import workloads as W
+    prob = W.decode128k() if args.workload == "decode128k" else W.decode32k()
+    threads = os.cpu_count() or 1
+    g = prob.n_heads // prob.n_kv_heads
+    rows = min(prob.rows, max(g, threads))
+    # size the per-step sample so that warm-up + steps take about two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    probe_keys = max(1024, prob.n // 64)
+    t_probe, _ = oracle_sample(prob, prob.q, probe_keys, rows, threads)
+    keys = int(min(prob.n, max(256, probe_keys * budget / max(t_probe, 1e-6))))
+    q_steps = prob.meta.get("q_steps")
+    for t in range(args.warmup):
+        oracle_sample(prob, prob.q if q_steps is None else q_steps[t % len(q_steps)], keys, rows,
+                      threads)
+    total, done = 0.0, 0
+    for t in range(args.steps):
+        secs, r = oracle_sample(prob, prob.q if q_steps is None else q_steps[t % len(q_steps)],
+                                keys, rows, threads)
+        total += secs
+        done += r
+    value = done * (keys / prob.n) / total
+    sample = (f"{rows} query heads per step over the first {keys} of n={prob.n} keys; value scaled "
+              f"by {keys}/{prob.n} (work is ~linear in n, the per-row sort n log n, so the "
+              f"scaling slightly favours the oracle)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload} (fp64 CPU oracle)", "eps": prob.eps},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("libcta", "reference"), default="libcta")
+    ap.add_argument("--workload", choices=("decode128k", "decode32k"), default="decode128k")
+    ap.add_argument("--eps", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--secondary", choices=("decode32k", "none"), default="decode32k",
+                    help="also measure this workload (same method, fewer steps) and nest it")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_libcta(args, rank, world, local_rank)
+        if res is not None and args.secondary != "none" and args.secondary != args.workload \
+                and world == 1:
+            sub = argparse.Namespace(**{**vars(args), "workload": args.secondary,
+                                        "steps": max(100, args.steps // 4)})
+            r2 = run_libcta(sub, rank, world, local_rank)
+            res["secondary"] = {k: r2[k] for k in ("value", "ms_per_step", "config", "roofline",
+                                                   "step_roofline", "phase_ms", "k_over_n_mean")}
+        if res is not None and world == 1 and not args.no_cpu_baseline:
+            from certified_top_sparse_b200 import workloads as W
+            prob = W.decode128k() if args.workload == "decode128k" else W.decode32k()
+            res["cpu_baseline"] = cpu_baseline(prob)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -10,8 +10,15 @@ Tolerances (the stated targets of the build, in writing):
     Exempt rows that differ must still be valid: GPU TV <= eps, and the GPU
     set differs from the oracle's by a few boundary keys.  Counts of class M
     at 1e-6 / 1e-7 / 1e-8 / 1e-9 and of class T are reported.
-  * out: per row ||out_gpu - out_ref||_inf <= tol * ||out_ref||_inf with
-    tol = 1e-5 (fp32 inputs) or 3e-3 (bf16 inputs and output).
+  * out, fp32: per row ||out_gpu - out_ref||_inf <= 1e-5 ||out_ref||_inf.
+  * out, bf16: compared in the output precision.  Rounding to bf16 (8
+    significant bits) alone moves a value by up to 2^-8 = 3.9e-3 relative,
+    more than a 3e-3 budget, so the GPU's bf16 output must equal the oracle's
+    fp64 output rounded to bf16, except where that value lies within
+    1e-5 * ||out_ref||_inf of a bf16 rounding midpoint (there the other
+    neighbour is allowed).  This checks the pre-rounding value to 1e-5 of the
+    row scale - tighter than 3e-3 - and the per-row relative error is also
+    reported.
   * TV and KL: within 1e-6 absolute.
   * err: |err_gpu - err_ref| <= 1e-4 err_ref + 1e-7.
 """
@@ -26,8 +33,10 @@ from certified_top_sparse_b200 import workloads as W
 WINDOWS = (1e-6, 1e-7, 1e-8, 1e-9)
 
 
-def out_tol(prob: W.Problem) -> float:
-    return 1e-5 if prob.q.dtype == torch.float32 else 3e-3
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """fp64 -> nearest bf16 (round to nearest even), returned as fp64."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64)).to(torch.bfloat16) \
+        .double().numpy()
 
 
 def oracle_dtype(prob: W.Problem) -> int:
@@ -71,6 +80,27 @@ def to_host(res: dict) -> dict:
     return h
 
 
+def check_out(og: np.ndarray, oo: np.ndarray, dtype: torch.dtype):
+    """Output check of the module docstring; og, oo are [rows, d] fp64.
+    Returns the per-row relative errors and the count of bf16 outputs that
+    took the other rounding neighbour."""
+    scale = np.abs(oo).max(axis=1)
+    rel = np.abs(og - oo).max(axis=1) / np.maximum(scale, 1e-30)
+    if dtype == torch.float32:
+        assert np.all(rel <= 1e-5), f"out rel err {rel.max()} > 1e-5"
+        return rel, 0
+    # arithmetic allowance before the final rounding: 1e-5 of the row scale
+    delta = 1e-5 * scale[:, None]
+    rounded = bf16_round(oo)
+    border = bf16_round(oo + delta) != bf16_round(oo - delta)
+    same = og == rounded
+    assert np.all(same | border), \
+        f"{int((~same & ~border).sum())} bf16 outputs differ from the rounded reference"
+    assert np.all(np.abs(og - oo) <= 2.0 ** -8 * np.abs(oo) + 1.01 * delta), \
+        "bf16 output off by more than rounding + 1e-5 of the row scale"
+    return rel, int((~same).sum())
+
+
 def compare(prob: W.Problem, eps: float, gpu: dict, ora: dict, rows=None, window: float = 1e-6):
     """Compare host copies of GPU results (rows `rows` of the GPU arrays, or
     all) with an oracle run over the same rows.  Returns a report dict;
@@ -80,7 +110,6 @@ def compare(prob: W.Problem, eps: float, gpu: dict, ora: dict, rows=None, window
     kg = gpu["k"][rows].astype(np.int64)
     ko = ora["k"].astype(np.int64)
     nrow = len(rows)
-    tol = out_tol(prob)
     classM = {w: (np.abs(ora["tv"] - eps) <= w) | (np.abs(ora["tv_km1"] - eps) <= w)
               for w in WINDOWS}
     classT = np.nan_to_num(ora["gap_u"], nan=np.inf) <= np.nan_to_num(ora["tie_bound"], nan=-1.0)
@@ -109,11 +138,7 @@ def compare(prob: W.Problem, eps: float, gpu: dict, ora: dict, rows=None, window
         dkl = np.abs(gpu["kl"][rows][ex] - ora["kl"][ex])
         assert np.all(dkl <= 1e-6), f"KL off by {dkl.max()}"
     # outputs
-    og = gpu["out"][rows][ex]
-    oo = ora["out"][ex]
-    scale = np.abs(oo).max(axis=1)
-    rel = np.abs(og - oo).max(axis=1) / np.maximum(scale, 1e-30)
-    assert np.all(rel <= tol), f"out rel err {rel.max()} > {tol}"
+    rel, n_ulp = check_out(gpu["out"][rows][ex], ora["out"][ex], prob.q.dtype)
     # exact head-tail error
     if gpu.get("err") is not None:
         eg = gpu["err"][rows][ex].astype(np.float64)
@@ -123,6 +148,6 @@ def compare(prob: W.Problem, eps: float, gpu: dict, ora: dict, rows=None, window
     return {
         "rows": nrow, "exact": int(exact.sum()), "differing_exempt": int((~exact).sum()),
         "classM": {f"{w:g}": int(classM[w].sum()) for w in WINDOWS}, "classT": int(classT.sum()),
-        "max_out_rel": float(rel.max()) if len(rel) else 0.0,
+        "max_out_rel": float(rel.max()) if len(rel) else 0.0, "bf16_ulp_diffs": n_ulp,
         "max_tv_abs": float(dtv.max()) if len(dtv) else 0.0,
     }

@@ -15,7 +15,7 @@ import torch
 
 from certified_top_sparse_b200 import workloads as W
 import certified_top_sparse_b200 as cta
-from parity import compare, group_rows, run_oracle, sub_problem, to_host
+from parity import check_out, compare, group_rows, run_oracle, sub_problem, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -179,13 +179,11 @@ def test_dense_reference_matches_oracle():
         dev = torch.device("cuda")
         out = cta.cta_dense_attn(prob.q.to(dev), prob.K.to(dev), prob.V.to(dev))
         torch.cuda.synchronize()
-        og = out.float().reshape(prob.rows, -1).cpu().numpy()
+        og = out.float().reshape(prob.rows, -1).cpu().numpy().astype(np.float64)
         oo = oracle.dense_attn(W.raw_words(prob.q), W.raw_words(prob.K), W.raw_words(prob.V),
                                n_heads=prob.n_heads, n_kv_heads=prob.n_kv_heads,
                                dtype=oracle.F32 if prob.q.dtype == torch.float32 else oracle.BF16)
-        tol = 1e-5 if prob.q.dtype == torch.float32 else 3e-3
-        scale = np.abs(oo).max(axis=1, keepdims=True)
-        assert np.all(np.abs(og - oo) <= tol * scale)
+        check_out(og, oo, prob.q.dtype)
 
 
 def test_err_equals_distance_to_dense_fp32():
