@@ -6,6 +6,7 @@ build script (``build``) and the seeded synthetic workloads (``workloads``).
 """
 from ._lib import (  # noqa: F401
     CTA_BF16, CTA_F32, CTA_DEV_INTERNAL, CTA_DEV_NONFINITE, CtaError, EXPORTED, LIB_PATH,
-    cta_certified_topk_attn, cta_dense_attn, cta_status_string, cta_version, cta_workspace_size,
-    load,
+    CTA_ERR_TOO_LARGE, NOALLOC_SCRATCH_BYTES, cta_certified_topk_attn,
+    cta_certified_topk_attn_noalloc, cta_dense_attn, cta_status_string, cta_version,
+    cta_workspace_size, load,
 )

@@ -22,7 +22,9 @@ CTA_DEV_INTERNAL = 0x2
 
 # Entry points declared in include/cta.h; the CPU test checks each is exported.
 EXPORTED = ("cta_opts_init", "cta_workspace_size", "cta_certified_topk_attn", "cta_dense_attn",
-            "cta_status_string", "cta_version")
+            "cta_status_string", "cta_version", "cta_certified_topk_attn_noalloc")
+CTA_ERR_TOO_LARGE = -7
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class cta_opts(ctypes.Structure):
@@ -65,6 +67,8 @@ def load() -> ctypes.CDLL:
         lib.cta_certified_topk_attn.argtypes = [vp, vp, vp, i64, i32, i32, i32, dbl, vp, vp, vp, vp,
                                                 ctypes.POINTER(cta_opts)]
         lib.cta_certified_topk_attn.restype = i32
+        lib.cta_certified_topk_attn_noalloc.argtypes = lib.cta_certified_topk_attn.argtypes
+        lib.cta_certified_topk_attn_noalloc.restype = i32
         lib.cta_dense_attn.argtypes = [vp, vp, vp, i64, i32, i32, i32, vp, ctypes.POINTER(cta_opts)]
         lib.cta_dense_attn.restype = i32
         lib.cta_status_string.argtypes = [i32]
@@ -186,3 +190,18 @@ def cta_dense_attn(q, K, V, *, out=None, stream=None):
     if rc != CTA_OK:
         raise CtaError(rc, "cta_dense_attn")
     return out
+
+
+def cta_certified_topk_attn_noalloc(q, K, V, eps, *, out, k_out, idx_out, tv_out, err_out=None,
+                                    kl_out=None, status_dev=None, stream=None):
+    """The no-allocation entry point: the library's own fixed scratch replaces
+    the workspace.  Every output must be passed in (this wrapper allocates
+    nothing either).  See include/cta.h for its limits and ordering rules."""
+    batch, n_heads, m, d, n_kv_heads, n = _shape(q, K, V)
+    o = make_opts(batch=batch, m=m, dtype=_dtype_code(q), stream=_stream_handle(stream),
+                  err_out=err_out, kl_out=kl_out, status_dev=status_dev)
+    rc = load().cta_certified_topk_attn_noalloc(_ptr(q), _ptr(K), _ptr(V), n, d, n_heads,
+                                                n_kv_heads, float(eps), _ptr(out), _ptr(k_out),
+                                                _ptr(idx_out), _ptr(tv_out), ctypes.byref(o))
+    if rc != CTA_OK:
+        raise CtaError(rc, "cta_certified_topk_attn_noalloc")

@@ -187,6 +187,7 @@ const char* cta_status_string(int status) {
     case CTA_ERR_CUDA: return "a CUDA launch or runtime call failed";
     case CTA_ERR_NONFINITE: return "non-finite logit";
     case CTA_ERR_TIMEOUT: return "timeout";
+    case CTA_ERR_TOO_LARGE: return "problem needs more scratch than the no-allocation entry point holds (CTA_NOALLOC_SCRATCH_BYTES = 32 MiB)";
     default: return "unknown status";
   }
 }

@@ -48,7 +48,8 @@ typedef enum {
   CTA_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or too small     */
   CTA_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed           */
   CTA_ERR_NONFINITE = -5,   /* reserved for host-side reporting of bit 1      */
-  CTA_ERR_TIMEOUT = -6      /* reserved: no kernel in this library waits      */
+  CTA_ERR_TIMEOUT = -6,     /* reserved: no kernel in this library waits      */
+  CTA_ERR_TOO_LARGE = -7    /* needs more scratch than CTA_NOALLOC_SCRATCH_BYTES */
 } cta_status;
 
 /* Bits OR-ed into *cta_opts.status_dev by device code. */
@@ -123,6 +124,37 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
  */
 int cta_dense_attn(const void* q, const void* K, const void* V, int64_t n, int d, int n_heads,
                    int n_kv_heads, void* out, const cta_opts* opts);
+
+/*
+ * Certified Top-k attention without any device allocation.  The paper has no
+ * counterpart: this is a deployment variant of cta_certified_topk_attn.
+ *
+ * For callers that cannot call cudaMalloc (for example while a CUDA graph is
+ * being captured, inside runtimes that forbid allocation outside their own
+ * memory pool, or under a device-memory budget fixed at start-up) and so
+ * cannot pass a workspace.  Same arguments, layouts, results and status codes
+ * as cta_certified_topk_attn; opts->workspace and opts->workspace_bytes are
+ * ignored.  The scratch is a fixed array of CTA_NOALLOC_SCRATCH_BYTES inside
+ * the library (32 MiB: enough for the 32K and 128K decode workloads of this
+ * library; about 4 * batch * n_heads * m * n bytes plus small records are
+ * needed, see cta_workspace_size).  Larger problems return CTA_ERR_TOO_LARGE
+ * before anything is launched.
+ *
+ *   - The array takes 32 MiB of device memory on every GPU where the library's
+ *     module is loaded, until the process exits.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array: calls that may overlap on
+ *     the GPU (different streams without ordering, or several host threads)
+ *     race and corrupt each other's results.  Order them on one stream.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define CTA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int cta_certified_topk_attn_noalloc(const void* q, const void* K, const void* V, int64_t n, int d,
+                                    int n_heads, int n_kv_heads, double eps, void* out,
+                                    int32_t* k_out, int32_t* idx_out, float* tv_out,
+                                    const cta_opts* opts);
 
 /* Static text for a cta_status value. */
 const char* cta_status_string(int status);
