@@ -23,11 +23,12 @@ struct Plan {
   int tiles_score;      // ceil(gm / rt_score)
   int rt_out;           // rows per output-pass tile
   int tiles_out;        // ceil(gm / rt_out)
-  float scale;          // 1/sqrt(d), rounded to fp32
+  float scale2;         // log2(e)/sqrt(d), rounded to fp32: weights are 2^(-scale2 (M - u))
   float two_s;          // 2^mass_shift, the fixed-point scale of the masses
   int mass_shift;
   double eps;
   int want_err;         // 1: also accumulate the dropped keys' value rows
+  int sel_cluster;      // CTAs (a thread-block cluster) per row in the selection pass
 };
 
 // Per-row result of the selection pass.
@@ -46,6 +47,9 @@ struct Partial {
   double wh;                // sum of kept weights
   double wt;                // sum of dropped weights
 };
+
+constexpr float kBinsPerOctave = 64.0f;  // selection bins per halving of the weight
+constexpr int kBins = 2048;               // selection bins (32 octaves; the last one is open)
 
 // ---------------------------------------------------------------------------
 // order-preserving 32-bit key of an fp32 logit: a > b  <=>  key(a) > key(b)
@@ -72,11 +76,20 @@ __device__ __forceinline__ bool is_kept(uint32_t key, uint32_t idx, uint32_t kst
   return key > kstar || (key == kstar && idx <= istar);
 }
 
-// Softmax numerator relative to the row max, fp32.  Both subtraction and
-// product are rounded explicitly so that every kernel computes bit-identical
-// weights for the same logit.
-__device__ __forceinline__ float weight(float u, float M, float scale) {
-  return expf(__fmul_rn(__fsub_rn(u, M), scale));
+// Softmax numerator relative to the row max: w = 2^(-a) with
+// a = (M - u) * log2(e)/sqrt(d) >= 0, i.e. exp((u - M)/sqrt(d)).  The
+// subtraction and product are rounded explicitly so that every kernel computes
+// bit-identical exponents (and so weights and bins) for the same logit.
+__device__ __forceinline__ float weight_arg(float u, float M, float scale2) {
+  return __fmul_rn(__fsub_rn(M, u), scale2);
+}
+__device__ __forceinline__ float weight(float u, float M, float scale2) {
+  return exp2f(-weight_arg(u, M, scale2));
+}
+// Selection bin of a logit: floor(64 a), so bin b holds weights in
+// (2^-(b+1)/64, 2^-b/64] up to exp2f's rounding; non-finite values stay in range.
+__device__ __forceinline__ int weight_bin(float a) {
+  return (int)fminf(fmaxf(a * kBinsPerOctave, 0.0f), (float)(kBins - 1));
 }
 
 // Fixed-point mass of a weight (exact integer sums, order independent).

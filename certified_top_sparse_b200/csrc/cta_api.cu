@@ -30,7 +30,7 @@ int ceil_log2(int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t u, cmax, sel, acc, part, status, total;
+  size_t u, cmax, sel, choff, acc, part, status, total;
 };
 
 int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, double eps,
@@ -67,12 +67,17 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, d
   if (nchunks > kMaxChunks) return CTA_ERR_SHAPE;
   p->chunk = (int)chunk;
   p->nchunks = (int)nchunks;
-  p->scale = (float)(1.0 / sqrt((double)d));
+  p->scale2 = (float)(1.4426950408889634 / sqrt((double)d));  // log2(e)/sqrt(d)
   int s = 62 - ceil_log2(n);
   if (s > 52) s = 52;
   p->mass_shift = s;
   p->two_s = ldexpf(1.0f, s);
   p->eps = eps;
+  // Selection: split rows over a cluster of up to 8 CTAs until ~2 CTAs per SM
+  // are busy, keeping at least 4096 keys per CTA.
+  int cs = 1;
+  while (cs < 8 && rows * cs * 2 <= 2 * 148 && n / (cs * 2) >= 4096) cs *= 2;
+  p->sel_cluster = cs;
   return CTA_OK;
 }
 
@@ -82,7 +87,8 @@ Layout layout(const Plan& p) {
   L.u = off;      off = align256(off + sizeof(float) * (size_t)p.rows * (size_t)p.n);
   L.cmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks);
   L.sel = off;    off = align256(off + sizeof(RowSel) * (size_t)p.rows);
-  L.acc = off;    off = align256(off + sizeof(double) * (size_t)p.rows * p.nchunks * 2 * p.d);
+  L.choff = off;  off = align256(off + sizeof(uint32_t) * (size_t)p.rows * p.nchunks);
+  L.acc = off;    off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks * 2 * p.d);
   L.part = off;   off = align256(off + sizeof(Partial) * (size_t)p.rows * p.nchunks);
   L.status = off; off = align256(off + sizeof(uint32_t));
   L.total = off;
@@ -140,7 +146,8 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   float* u = reinterpret_cast<float*>(ws + L.u);
   float* cmax = reinterpret_cast<float*>(ws + L.cmax);
   RowSel* sel = reinterpret_cast<RowSel*>(ws + L.sel);
-  double* acc = reinterpret_cast<double*>(ws + L.acc);
+  uint32_t* choff = reinterpret_cast<uint32_t*>(ws + L.choff);
+  float* acc = reinterpret_cast<float*>(ws + L.acc);
   Partial* part = reinterpret_cast<Partial*>(ws + L.part);
   uint32_t* status = opts->status_dev ? opts->status_dev : reinterpret_cast<uint32_t*>(ws + L.status);
   cudaStream_t st = static_cast<cudaStream_t>(opts->stream);
@@ -149,10 +156,11 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
   if (launch_score(opts->dtype, q, K, u, cmax, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_select(u, cmax, sel, k_out, tv_out, idx_out, p, status, st) != cudaSuccess)
+  if (launch_select(u, cmax, sel, k_out, tv_out, choff, p, status, st) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_gather(opts->dtype, V, u, sel, acc, part, p, st) != cudaSuccess) return CTA_ERR_CUDA;
+  if (launch_gather(opts->dtype, V, u, sel, choff, idx_out, acc, part, p, st) != cudaSuccess)
+    return CTA_ERR_CUDA;
   if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
   if (launch_finalize(opts->dtype, sel, acc, part, out, opts->err_out, opts->kl_out, p, status, st) !=
       cudaSuccess)

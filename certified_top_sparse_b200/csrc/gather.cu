@@ -30,7 +30,8 @@ constexpr int kGUnroll = 4;
 template <typename T, int D, int RT, bool ERR>
 __global__ void __launch_bounds__(kGatherThreads)
 gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel* __restrict__ sel,
-              double* __restrict__ acc_out, Partial* __restrict__ part_out, Plan p) {
+              const uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out,
+              float* __restrict__ acc_out, Partial* __restrict__ part_out, Plan p) {
   constexpr int EPL = Elem<T>::EPL;
   constexpr int LPK = D / EPL;
   constexpr int KPI = kWarp / LPK;
@@ -67,7 +68,7 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
       const float* ur = u + (row0 + r) * p.n + key0;
       for (int i = threadIdx.x; i < nk; i += kGatherThreads) {
         const float x = ur[i];
-        const float w = weight(x, rs.M, p.scale);
+        const float w = weight(x, rs.M, p.scale2);
         const bool kept = is_kept(order_key(x), (uint32_t)(key0 + i), rs.kstar, (uint32_t)rs.istar);
         sw[r * p.chunk + i] = kept ? w : -w;
         if (kept) sh[r] += (double)w; else st[r] += (double)w;
@@ -93,6 +94,36 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
     pr.wh = a;
     pr.wt = b;
     part_out[(row0 + threadIdx.x) * p.nchunks + chunk] = pr;
+  }
+
+  // ---- the chunk's kept indices, ascending, at the offset from selection -----
+  {
+    __shared__ uint32_t wcount[kGatherWarps];
+    const int per = ((nk + kGatherThreads - 1) / kGatherThreads) * kWarp;  // keys per warp
+    const int k_lo = min(nk, warp * per), k_hi = min(nk, k_lo + per);
+    for (int r = 0; r < nrows; ++r) {
+      const float* swr = sw + r * p.chunk;
+      uint32_t cnt = 0u;
+      for (int k0 = k_lo; k0 < k_hi; k0 += kWarp) {
+        const int key = k0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, key < k_hi && !signbit(swr[key])));
+      }
+      if (lane == 0) wcount[warp] = cnt;
+      __syncthreads();
+      uint32_t off = chunk_off[(row0 + r) * p.nchunks + chunk];
+      for (int w = 0; w < warp; ++w) off += wcount[w];
+      for (int k0 = k_lo; k0 < k_hi; k0 += kWarp) {
+        const int key = k0 + lane;
+        const bool kept = key < k_hi && !signbit(swr[key]);
+        const uint32_t m = __ballot_sync(0xffffffffu, kept);
+        if (kept) {
+          const uint32_t at = off + __popc(m & ((1u << lane) - 1u));
+          if (at < (uint32_t)p.n) idx_out[(row0 + r) * p.n + at] = (int32_t)(key0 + key);
+        }
+        off += __popc(m);
+      }
+      __syncthreads();
+    }
   }
 
   // ---- step B: weighted value sums -------------------------------------------
@@ -155,13 +186,14 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
     if (r >= nrows) continue;
     double s = 0.0;
     for (int g = 0; g < SLOTS; ++g) s += (double)sred[((g * NACC + a) * RT + r) * D + dim];
-    acc_out[(((row0 + r) * p.nchunks + chunk) * 2 + a) * D + dim] = s;
+    acc_out[(((row0 + r) * p.nchunks + chunk) * 2 + a) * D + dim] = (float)s;
   }
 }
 
 template <typename T, int D, int RT, bool ERR>
-cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, double* acc,
-                            Partial* part, const Plan& p, cudaStream_t st) {
+cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel,
+                            const uint32_t* choff, int32_t* idx, float* acc, Partial* part,
+                            const Plan& p, cudaStream_t st) {
   constexpr int EPL = Elem<T>::EPL;
   constexpr int SLOTS = kGatherWarps * (kWarp / (D / EPL));
   const size_t smem = sizeof(float) * ((size_t)RT * p.chunk + (size_t)SLOTS * (ERR ? 2 : 1) * RT * D);
@@ -169,46 +201,69 @@ cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, do
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.tiles_out, p.nchunks, p.groups);
-  kern<<<grid, kGatherThreads, smem, st>>>(static_cast<const T*>(V), u, sel, acc, part, p);
+  kern<<<grid, kGatherThreads, smem, st>>>(static_cast<const T*>(V), u, sel, choff, idx, acc, part,
+                                           p);
   return cudaGetLastError();
 }
 
 template <typename T, int D, bool ERR>
-cudaError_t launch_gather_e(const void* V, const float* u, const RowSel* sel, double* acc,
-                            Partial* part, const Plan& p, cudaStream_t st) {
+cudaError_t launch_gather_e(const void* V, const float* u, const RowSel* sel,
+                            const uint32_t* choff, int32_t* idx, float* acc, Partial* part,
+                            const Plan& p, cudaStream_t st) {
   switch (p.rt_out) {
-    case 1: return launch_gather_t<T, D, 1, ERR>(V, u, sel, acc, part, p, st);
-    case 2: return launch_gather_t<T, D, 2, ERR>(V, u, sel, acc, part, p, st);
-    case 4: return launch_gather_t<T, D, 4, ERR>(V, u, sel, acc, part, p, st);
+    case 1: return launch_gather_t<T, D, 1, ERR>(V, u, sel, choff, idx, acc, part, p, st);
+    case 2: return launch_gather_t<T, D, 2, ERR>(V, u, sel, choff, idx, acc, part, p, st);
+    case 4: return launch_gather_t<T, D, 4, ERR>(V, u, sel, choff, idx, acc, part, p, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_gather_d(const void* V, const float* u, const RowSel* sel, double* acc,
-                            Partial* part, const Plan& p, cudaStream_t st) {
-  return p.want_err ? launch_gather_e<T, D, true>(V, u, sel, acc, part, p, st)
-                    : launch_gather_e<T, D, false>(V, u, sel, acc, part, p, st);
+cudaError_t launch_gather_d(const void* V, const float* u, const RowSel* sel,
+                            const uint32_t* choff, int32_t* idx, float* acc, Partial* part,
+                            const Plan& p, cudaStream_t st) {
+  return p.want_err ? launch_gather_e<T, D, true>(V, u, sel, choff, idx, acc, part, p, st)
+                    : launch_gather_e<T, D, false>(V, u, sel, choff, idx, acc, part, p, st);
 }
 
 // ---- phase 4 ------------------------------------------------------------------
 
+constexpr int kFinThreads = 256;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
-finalize_kernel(const RowSel* __restrict__ sel, const double* __restrict__ acc,
+__global__ void __launch_bounds__(kFinThreads)
+finalize_kernel(const RowSel* __restrict__ sel, const float* __restrict__ acc,
                 const Partial* __restrict__ part, T* __restrict__ out, float* __restrict__ err_out,
                 float* __restrict__ kl_out, Plan p, uint32_t* __restrict__ status) {
+  constexpr int G = kFinThreads / D;   // thread groups, each over every G-th chunk
+  __shared__ double s_ah[G][D], s_at[G][D], s_w[G][2];
   __shared__ double red[D / 32];
   const int64_t row = blockIdx.x;
-  const int dim = threadIdx.x;
+  const int dim = threadIdx.x % D;
+  const int grp = threadIdx.x / D;
   double ah = 0.0, at = 0.0, wh = 0.0, wt = 0.0;
-  for (int c = 0; c < p.nchunks; ++c) {
-    const double* a = acc + ((row * p.nchunks + c) * 2) * D;
-    ah += a[dim];
-    if (p.want_err) at += a[D + dim];
-    const Partial pr = part[row * p.nchunks + c];
-    wh += pr.wh;
-    wt += pr.wt;
+  const float* a = acc + row * p.nchunks * 2 * D + dim;
+#pragma unroll 4
+  for (int c = grp; c < p.nchunks; c += G) {
+    ah += a[(int64_t)c * 2 * D];
+    if (p.want_err) at += a[(int64_t)c * 2 * D + D];
+    if (dim == 0) {
+      const Partial pr = part[row * p.nchunks + c];
+      wh += pr.wh;
+      wt += pr.wt;
+    }
+  }
+  s_ah[grp][dim] = ah;
+  s_at[grp][dim] = at;
+  if (dim == 0) { s_w[grp][0] = wh; s_w[grp][1] = wt; }
+  __syncthreads();
+  if (threadIdx.x >= D) return;
+  ah = 0.0; at = 0.0; wh = 0.0; wt = 0.0;
+  for (int g = 0; g < G; ++g) {  // fixed order
+    ah += s_ah[g][dim];
+    at += s_at[g][dim];
+    wh += s_w[g][0];
+    wt += s_w[g][1];
   }
   const double mu_h = ah / wh;
   Elem<T>::store1(out + row * D + dim, (float)mu_h);
@@ -219,7 +274,7 @@ finalize_kernel(const RowSel* __restrict__ sel, const double* __restrict__ acc,
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if ((dim & 31) == 0) red[dim >> 5] = s;
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;" ::"r"(D));  // the first D threads only
     if (dim == 0) {
       double tot = 0.0;
       for (int w = 0; w < D / 32; ++w) tot += red[w];
@@ -231,30 +286,31 @@ finalize_kernel(const RowSel* __restrict__ sel, const double* __restrict__ acc,
 }
 
 template <typename T>
-cudaError_t launch_finalize_t(const RowSel* sel, const double* acc, const Partial* part, void* out,
+cudaError_t launch_finalize_t(const RowSel* sel, const float* acc, const Partial* part, void* out,
                               float* err_out, float* kl_out, const Plan& p, uint32_t* status,
                               cudaStream_t st) {
   if (p.d == 64)
-    finalize_kernel<T, 64><<<(unsigned)p.rows, 64, 0, st>>>(sel, acc, part, static_cast<T*>(out),
-                                                            err_out, kl_out, p, status);
+    finalize_kernel<T, 64><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
+        sel, acc, part, static_cast<T*>(out), err_out, kl_out, p, status);
   else
-    finalize_kernel<T, 128><<<(unsigned)p.rows, 128, 0, st>>>(sel, acc, part, static_cast<T*>(out),
-                                                              err_out, kl_out, p, status);
+    finalize_kernel<T, 128><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
+        sel, acc, part, static_cast<T*>(out), err_out, kl_out, p, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, double* acc,
-                          Partial* part, const Plan& p, cudaStream_t st) {
+cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel,
+                          const uint32_t* choff, int32_t* idx, float* acc, Partial* part,
+                          const Plan& p, cudaStream_t st) {
   if (dtype == kDtypeF32)
-    return p.d == 64 ? launch_gather_d<float, 64>(V, u, sel, acc, part, p, st)
-                     : launch_gather_d<float, 128>(V, u, sel, acc, part, p, st);
-  return p.d == 64 ? launch_gather_d<__nv_bfloat16, 64>(V, u, sel, acc, part, p, st)
-                   : launch_gather_d<__nv_bfloat16, 128>(V, u, sel, acc, part, p, st);
+    return p.d == 64 ? launch_gather_d<float, 64>(V, u, sel, choff, idx, acc, part, p, st)
+                     : launch_gather_d<float, 128>(V, u, sel, choff, idx, acc, part, p, st);
+  return p.d == 64 ? launch_gather_d<__nv_bfloat16, 64>(V, u, sel, choff, idx, acc, part, p, st)
+                   : launch_gather_d<__nv_bfloat16, 128>(V, u, sel, choff, idx, acc, part, p, st);
 }
 
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const double* acc, const Partial* part,
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const Partial* part,
                             void* out, float* err_out, float* kl_out, const Plan& p,
                             uint32_t* status, cudaStream_t st) {
   if (dtype == kDtypeF32)

@@ -16,17 +16,20 @@ constexpr int kDtypeBF16 = CTA_BF16;
 cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, float* cmax,
                          const Plan& p, uint32_t* status, cudaStream_t st);
 
-// Phase 2: per-row certified selection; writes sel, k_out, tv_out and idx_out.
+// Phase 2: per-row certified selection; writes sel, k_out, tv_out and, per
+// (row, chunk), the offset of the chunk's first kept index (chunk_off).
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
-                          float* tv_out, int32_t* idx_out, const Plan& p, uint32_t* status,
+                          float* tv_out, uint32_t* chunk_off, const Plan& p, uint32_t* status,
                           cudaStream_t st);
 
-// Phase 3: per-(tile, chunk) weighted value sums of kept (and dropped) keys.
+// Phase 3: per-(tile, chunk) weighted value sums of kept (and dropped) keys
+// and the chunk's kept indices, written into idx_out at chunk_off.
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel,
-                          double* acc, Partial* part, const Plan& p, cudaStream_t st);
+                          const uint32_t* chunk_off, int32_t* idx_out, float* acc, Partial* part,
+                          const Plan& p, cudaStream_t st);
 
 // Phase 4: combine chunk partials into out, err, kl.
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const double* acc, const Partial* part,
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const Partial* part,
                             void* out, float* err_out, float* kl_out, const Plan& p,
                             uint32_t* status, cudaStream_t st);
 
