@@ -19,6 +19,7 @@ CTA_F32, CTA_BF16 = 0, 1
 CTA_OK = 0
 CTA_DEV_NONFINITE = 0x1
 CTA_DEV_INTERNAL = 0x2
+CTA_DEV_TIMEOUT = 0x4
 
 # Entry points declared in include/cta.h; the CPU test checks each is exported.
 EXPORTED = ("cta_opts_init", "cta_workspace_size", "cta_certified_topk_attn", "cta_dense_attn",

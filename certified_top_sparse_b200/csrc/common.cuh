@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 namespace cta {
 
@@ -165,27 +166,133 @@ template <> struct Elem<__nv_bfloat16> {
 };
 
 // ---------------------------------------------------------------------------
-// Transposed butterfly reduction across the LPK lanes that share one key.
-// On entry each lane holds CNT partial sums (one per row of a tile); on exit
-// a[0] holds the full sum of row (lane % LPK) / (LPK / CNT).  Uses
-// CNT - 1 + log2(LPK / CNT) shuffles instead of CNT * log2(LPK).
+// Packed fp32 pair FMA (Blackwell f32x2): d = a * b + c on both lanes, each
+// with a single IEEE round-to-nearest like fmaf.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n"
+      " mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// The same on packed pairs held in 64-bit registers (no repacking per FMA).
+__device__ __forceinline__ unsigned long long fma2p(unsigned long long a, unsigned long long b,
+                                                    unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long pack2(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ float sum2(unsigned long long v) {
+  float x, y;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(v));
+  return x + y;
+}
+
+// bf16 pair (one 32-bit word, element 0 in the low half) widened to fp32.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk-copy (TMA, non-multicast) helpers.  Every wait is bounded
+// by wall time: on expiry it reports failure instead of spinning forever.
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// Wait for the phase with the given parity to complete; false after ~2 s.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing on bar.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes,
+                                          unsigned long long* bar, unsigned long long policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Transposed butterfly reduction across the LPK lanes that share one key,
+// without selects.  Each lane holds CNT partial sums, slot s holding row
+// s ^ mask where mask = row_mask<CNT, LPK>(part), part = lane % LPK (the
+// caller arranges its rows that way).  At the level with xor offset O the two
+// partner lanes differ in the mask bit of that level, so the row a lane keeps
+// is always in its low half and the row its partner needs is always in its
+// high half: a[i] += shfl_xor(a[i + H], O).  On exit a[0..max(1, CNT/LPK))
+// hold full sums of rows i ^ mask, i.e. row part / (LPK / CNT) when
+// CNT <= LPK and rows i + (CNT / LPK) * part otherwise.
+template <int CNT, int LPK>
+__device__ __forceinline__ int row_mask(int part) {
+  if constexpr (CNT >= LPK) {
+    return (CNT / LPK) * part;
+  } else {
+    int shift = 0;
+    while ((LPK >> shift) > CNT) ++shift;  // log2(LPK / CNT)
+    return part >> shift;
+  }
+}
+
 template <int CNT, int O>
-struct TransposeReduce {
-  __device__ __forceinline__ static void run(float* a, int lane) {
+struct XorReduce {
+  __device__ __forceinline__ static void run(float* a) {
     if constexpr (O >= 1) {
       if constexpr (CNT > 1) {
         constexpr int H = CNT / 2;
-        const bool upper = (lane & O) != 0;
 #pragma unroll
-        for (int i = 0; i < H; ++i) {
-          const float send = upper ? a[i] : a[i + H];
-          const float keep = upper ? a[i + H] : a[i];
-          a[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
-        }
-        TransposeReduce<H, O / 2>::run(a, lane);
+        for (int i = 0; i < H; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[i + H], O);
+        XorReduce<H, O / 2>::run(a);
       } else {
         a[0] += __shfl_xor_sync(0xffffffffu, a[0], O);
-        TransposeReduce<1, O / 2>::run(a, lane);
+        XorReduce<1, O / 2>::run(a);
       }
     }
   }

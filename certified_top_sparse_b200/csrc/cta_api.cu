@@ -33,8 +33,8 @@ struct Layout {
   size_t u, cmax, sel, choff, acc, part, status, total;
 };
 
-int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, double eps,
-              Plan* p) {
+int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, int dtype,
+              double eps, Plan* p) {
   if (d != 64 && d != 128) return CTA_ERR_SHAPE;
   if (n < 1 || n > kMaxN) return CTA_ERR_SHAPE;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return CTA_ERR_SHAPE;
@@ -50,7 +50,9 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, d
   p->d = d;
   p->gm = (int)gm;
   p->groups = (int)groups;
-  p->rt_score = next_pow2((int)(gm < 8 ? gm : 8));
+  // Rows per score tile: 8 for fp32, 4 for bf16 (register budget of 2 CTAs/SM).
+  const int rt_max = (dtype == CTA_F32) ? 8 : 4;
+  p->rt_score = next_pow2((int)(gm < rt_max ? gm : rt_max));
   p->tiles_score = (int)((gm + p->rt_score - 1) / p->rt_score);
   p->rt_out = next_pow2((int)(gm < 4 ? gm : 4));
   p->tiles_out = (int)((gm + p->rt_out - 1) / p->rt_out);
@@ -122,7 +124,7 @@ size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const c
   cta_opts_init(&def);
   if (!o) o = &def;
   Plan p;
-  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, 0.5, &p) != CTA_OK) return 0;
+  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, o->dtype, 0.5, &p) != CTA_OK) return 0;
   return layout(p).total;
 }
 
@@ -135,7 +137,7 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
   if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return CTA_ERR_ARG;
   Plan p;
-  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, eps, &p);
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps, &p);
   if (rc != CTA_OK) return rc;
   p.want_err = opts->err_out != nullptr;
   const Layout L = layout(p);
@@ -178,7 +180,7 @@ int cta_dense_attn(const void* q, const void* K, const void* V, int64_t n, int d
   if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
   if (!aligned16(q) || !aligned16(K) || !aligned16(V)) return CTA_ERR_ARG;
   Plan p;
-  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, 0.5, &p);
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, 0.5, &p);
   if (rc != CTA_OK) return rc;
   if (launch_dense(opts->dtype, q, K, V, out, n, d, p.rows, p.gm,
                    static_cast<cudaStream_t>(opts->stream)) != cudaSuccess)

@@ -48,13 +48,14 @@ typedef enum {
   CTA_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or too small     */
   CTA_ERR_CUDA = -4,        /* a CUDA launch or runtime call failed           */
   CTA_ERR_NONFINITE = -5,   /* reserved for host-side reporting of bit 1      */
-  CTA_ERR_TIMEOUT = -6,     /* reserved: no kernel in this library waits      */
+  CTA_ERR_TIMEOUT = -6,     /* reserved for host-side reporting of bit 4      */
   CTA_ERR_TOO_LARGE = -7    /* needs more scratch than CTA_NOALLOC_SCRATCH_BYTES */
 } cta_status;
 
 /* Bits OR-ed into *cta_opts.status_dev by device code. */
 #define CTA_DEV_NONFINITE 0x1u  /* a logit was NaN or infinite: outputs of that row are meaningless */
 #define CTA_DEV_INTERNAL 0x2u   /* an internal consistency check failed (a library bug)            */
+#define CTA_DEV_TIMEOUT 0x4u    /* a pipeline wait in a kernel gave up after ~2 s (results invalid) */
 
 /* Optional arguments.  Initialise with cta_opts_init() and override fields. */
 typedef struct {
