@@ -14,6 +14,7 @@ constexpr int kWarp = 32;
 // Launch plan, computed once on the host per call and passed by value.
 struct Plan {
   int64_t n;            // keys per KV head
+  int64_t ustride;      // row stride of the logit buffer: n rounded up to 64
   int64_t rows;         // batch * n_heads * m
   int d;                // head dimension
   int gm;               // rows sharing one KV head: (n_heads / n_kv_heads) * m
@@ -30,6 +31,8 @@ struct Plan {
   double eps;
   int want_err;         // 1: also accumulate the dropped keys' value rows
   int sel_cluster;      // CTAs (a thread-block cluster) per row in the selection pass
+  int nranges;          // output pass: chunk ranges per (KV group, row tile)
+  int range_len;        // chunks per range
 };
 
 // Per-row result of the selection pass.
@@ -41,12 +44,8 @@ struct RowSel {
   unsigned long long Z;     // total fixed-point mass
   unsigned long long C;     // kept fixed-point mass
   double tv;                // (Z - C) / Z
-};
-
-// Per (row, chunk) record of the output pass.
-struct Partial {
-  double wh;                // sum of kept weights
-  double wt;                // sum of dropped weights
+  double wh;                // sum of the kept keys' weights (fp64, fixed order)
+  double wt;                // sum of the dropped keys' weights
 };
 
 constexpr float kBinsPerOctave = 64.0f;  // selection bins per halving of the weight

@@ -30,8 +30,20 @@ int ceil_log2(int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t u, cmax, sel, choff, acc, part, status, total;
+  size_t u, cmax, sel, choff, acc, status, total;
 };
+
+// Output pass: each CTA owns a contiguous range of chunks of one (group, row
+// tile); ranges are cut so that the ranges of all units about fill ctas_per_sm
+// CTAs on every SM.
+void set_ranges(Plan* p, int ctas_per_sm) {
+  const int64_t units_out = (int64_t)p->groups * p->tiles_out;
+  int64_t nr = ((int64_t)ctas_per_sm * 148 + units_out - 1) / units_out;
+  if (nr > p->nchunks) nr = p->nchunks;
+  if (nr < 1) nr = 1;
+  p->range_len = (int)((p->nchunks + nr - 1) / nr);
+  p->nranges = (int)((p->nchunks + p->range_len - 1) / p->range_len);
+}
 
 int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, int dtype,
               double eps, Plan* p) {
@@ -46,6 +58,7 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   if (gm > (1 << 24) || rows > INT32_MAX || groups > 65535) return CTA_ERR_SHAPE;
   memset(p, 0, sizeof(*p));
   p->n = n;
+  p->ustride = (n + 63) & ~(int64_t)63;  // 256-byte aligned rows for the bulk copies
   p->rows = rows;
   p->d = d;
   p->gm = (int)gm;
@@ -80,18 +93,18 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   int cs = 1;
   while (cs < 8 && rows * cs * 2 <= 2 * 148 && n / (cs * 2) >= 4096) cs *= 2;
   p->sel_cluster = cs;
+  set_ranges(p, 2);
   return CTA_OK;
 }
 
 Layout layout(const Plan& p) {
   Layout L;
   size_t off = 0;
-  L.u = off;      off = align256(off + sizeof(float) * (size_t)p.rows * (size_t)p.n);
+  L.u = off;      off = align256(off + sizeof(float) * (size_t)p.rows * (size_t)p.ustride);
   L.cmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks);
   L.sel = off;    off = align256(off + sizeof(RowSel) * (size_t)p.rows);
   L.choff = off;  off = align256(off + sizeof(uint32_t) * (size_t)p.rows * p.nchunks);
   L.acc = off;    off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks * 2 * p.d);
-  L.part = off;   off = align256(off + sizeof(Partial) * (size_t)p.rows * p.nchunks);
   L.status = off; off = align256(off + sizeof(uint32_t));
   L.total = off;
   return L;
@@ -140,6 +153,7 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps, &p);
   if (rc != CTA_OK) return rc;
   p.want_err = opts->err_out != nullptr;
+  set_ranges(&p, gather_ctas_per_sm(p.want_err));
   const Layout L = layout(p);
   if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
     return CTA_ERR_WORKSPACE;
@@ -150,7 +164,6 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   RowSel* sel = reinterpret_cast<RowSel*>(ws + L.sel);
   uint32_t* choff = reinterpret_cast<uint32_t*>(ws + L.choff);
   float* acc = reinterpret_cast<float*>(ws + L.acc);
-  Partial* part = reinterpret_cast<Partial*>(ws + L.part);
   uint32_t* status = opts->status_dev ? opts->status_dev : reinterpret_cast<uint32_t*>(ws + L.status);
   cudaStream_t st = static_cast<cudaStream_t>(opts->stream);
   void** ev = opts->phase_events;
@@ -158,13 +171,13 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
   if (launch_score(opts->dtype, q, K, u, cmax, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_select(u, cmax, sel, k_out, tv_out, choff, p, status, st) != cudaSuccess)
+  if (launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, p, status, st) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_gather(opts->dtype, V, u, sel, choff, idx_out, acc, part, p, st) != cudaSuccess)
+  if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_finalize(opts->dtype, sel, acc, part, out, opts->err_out, opts->kl_out, p, status, st) !=
+  if (launch_finalize(opts->dtype, sel, acc, out, opts->err_out, opts->kl_out, p, status, st) !=
       cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;

@@ -16,22 +16,22 @@ constexpr int kDtypeBF16 = CTA_BF16;
 cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, float* cmax,
                          const Plan& p, uint32_t* status, cudaStream_t st);
 
-// Phase 2: per-row certified selection; writes sel, k_out, tv_out and, per
-// (row, chunk), the offset of the chunk's first kept index (chunk_off).
+// Phase 2: per-row certified selection; writes sel, k_out, tv_out and the
+// kept indices (idx_out), using chunk_off as its per-chunk offset scratch.
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
-                          float* tv_out, uint32_t* chunk_off, const Plan& p, uint32_t* status,
-                          cudaStream_t st);
+                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, const Plan& p,
+                          uint32_t* status, cudaStream_t st);
 
-// Phase 3: per-(tile, chunk) weighted value sums of kept (and dropped) keys
-// and the chunk's kept indices, written into idx_out at chunk_off.
+// Phase 3: per-(row, chunk range) weighted value sums of kept (and dropped)
+// keys.  gather_ctas_per_sm: the CTAs per SM its launch is planned for.
+int gather_ctas_per_sm(bool want_err);
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel,
-                          const uint32_t* chunk_off, int32_t* idx_out, float* acc, Partial* part,
-                          const Plan& p, cudaStream_t st);
+                          float* acc, const Plan& p, uint32_t* status, cudaStream_t st);
 
 // Phase 4: combine chunk partials into out, err, kl.
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const Partial* part,
-                            void* out, float* err_out, float* kl_out, const Plan& p,
-                            uint32_t* status, cudaStream_t st);
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, void* out,
+                            float* err_out, float* kl_out, const Plan& p, uint32_t* status,
+                            cudaStream_t st);
 
 // Dense reference attention (all keys, fp32 online softmax).
 cudaError_t launch_dense(int dtype, const void* q, const void* K, const void* V, void* out,

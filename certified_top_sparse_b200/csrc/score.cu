@@ -244,7 +244,7 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
     for (int r = 0; r < RT; ++r) {
       mx[r] = kNegInf;
       if (r < nrows) {
-        float* dst = u + (row0 + r) * p.n + key0;
+        float* dst = u + (row0 + r) * p.ustride + key0;
         for (int i = threadIdx.x; i < nk; i += kScoreThreads) {
           const float x = su[r * su_stride + i];
           dst[i] = x;

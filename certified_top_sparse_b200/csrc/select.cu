@@ -25,8 +25,12 @@
 //      bin, still an interval of the ranking), finds the sub-bin that holds
 //      the cut and sorts only its keys (logit desc, index asc); a prefix sum
 //      of their exact masses gives the last kept key (K*, I*) and k_eps.
-//   5. Per output chunk, the exclusive offset of its first kept index (the
-//      output pass writes the kept indices with it).
+//   5. Per output chunk, the exclusive offset of its first kept index.
+//   6. Each CTA writes the kept indices of its segment, ascending, from those
+//      offsets (one warp per chunk, ballots of 32 keys).
+// Alongside, the fp64 sums of the kept and of the dropped weights (the output
+// normalisers): pass 3 sums the keys above and below the window, CTA 0 splits
+// the window's candidates at the cut; every reduction has a fixed order.
 // A window with more than 4096 keys (near-ties, e.g. all-equal logits) is
 // first narrowed exactly by 8-bit radix digits of the composite key (logit
 // order, then index); then the per-chunk counts come from a recount pass.
@@ -48,6 +52,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kSubPerBin = 64;          // sub-bins per bin: 4096 per halving of the weight
 constexpr int kSub = 2048;              // sub-bins available (a window of up to 32 bins)
 constexpr int kLocalChunks = 1024;      // per-CTA chunk counters kept in shared memory
+constexpr int kIdxBatch = 8;            // 32-key words in flight per warp in the index pass
 constexpr int kBinsPerThread = kBins / kSelThreads;
 constexpr double kBoundSlack = 4e-6;    // covers exp2f's error (2 ulp) with margin
 constexpr double kDecideSlack = 1e-9;   // covers fp64 rounding in the exact test
@@ -67,6 +72,9 @@ struct SelShared {
   unsigned long long dmass[256];    // radix narrowing: digit masses (this CTA)
   unsigned int dcnt[256];           //                  digit counts (this CTA)
   unsigned long long warp_buf[kSelWarps];
+  double fwarp[kSelWarps][2];       // per-warp fp64 sums
+  double fpart[2];                  // this CTA's fp64 weight sums: kept (above), dropped (below)
+  double fsum[2];                   // block result of block_sum2
   unsigned long long zpart, tpart, wpart;  // this CTA's exact masses: all, below, window
   unsigned long long Z, T, Wn;      // the row's, summed over the cluster
   unsigned long long local_kept;    // kept keys in this CTA's segment (read by the cluster)
@@ -114,6 +122,25 @@ __device__ unsigned long long block_sum(unsigned long long v, SelShared& S) {
   unsigned long long t;
   block_scan_excl(v, &t, S);
   return t;
+}
+
+// Fixed-order block sums of two fp64 values per thread (into S.fsum).
+__device__ void block_sum2(double a, double b, SelShared& S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  if (lane == 0) { S.fwarp[warp][0] = a; S.fwarp[warp][1] = b; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double x = 0.0, y = 0.0;
+    for (int w = 0; w < kSelWarps; ++w) { x += S.fwarp[w][0]; y += S.fwarp[w][1]; }
+    S.fsum[0] = x;
+    S.fsum[1] = y;
+  }
+  __syncthreads();
 }
 
 __device__ float block_max(float v, SelShared& S) {
@@ -213,7 +240,8 @@ __device__ __forceinline__ unsigned long long bin_mass_lo(int b, int shift) {
 __global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSel* __restrict__ sel,
               int32_t* __restrict__ k_out, float* __restrict__ tv_out,
-              uint32_t* __restrict__ chunk_off, Plan p, uint32_t* __restrict__ status) {
+              uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out, Plan p,
+              uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
@@ -226,7 +254,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   const int warp = tid >> 5;
   const int64_t row = blockIdx.x / CS;
   const int64_t n = p.n;
-  const float* ur = u + row * n;
+  const float* ur = u + row * p.ustride;
   // Segments are whole output chunks, so a chunk's count has one owner CTA.
   const int64_t seg = (((n + CS - 1) / CS + p.chunk - 1) / p.chunk) * p.chunk;
   const int64_t lo = min(n, (int64_t)rank * seg);
@@ -341,16 +369,19 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   // ---- 3. exact masses, candidates, certainly-kept counts per chunk -----------
   {
     unsigned long long z = 0ull, t = 0ull, wn = 0ull;
+    double fa = 0.0, fb = 0.0;  // fp64 weight sums above / below the window
     for_each_quad<4>(ur, lo, hi, vec, [&](const float* x, int64_t i, const bool* ok) {
       unsigned int above = 0u;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float a = weight_arg(x[e], M, s2);
         const int b = weight_bin(a);
-        const unsigned long long W = ok[e] ? fixed_mass(exp2f(-a), two_s) : 0ull;
+        const float w = ok[e] ? exp2f(-a) : 0.0f;
+        const unsigned long long W = fixed_mass(w, two_s);
         z += W;
-        if (b > b2) t += W;
+        if (b > b2) { t += W; fb += (double)w; }
         else if (b >= b1) wn += W;
+        else fa += (double)w;
         if (direct && ok[e]) {
           if (b < b1) ++above;
           else if (b <= b2) {
@@ -376,7 +407,8 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       atomicAdd(&S.tpart, t);
       atomicAdd(&S.wpart, wn);
     }
-    __syncthreads();
+    block_sum2(fa, fb, S);
+    if (tid == 0) { S.fpart[0] = S.fsum[0]; S.fpart[1] = S.fsum[1]; }
     if (direct && local_cc)
       for (int c = c0 + tid; c < c1; c += kSelThreads) cc[c] = S.lcc[c - c0];
   }
@@ -495,6 +527,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
     unsigned long long* srt = S.cand;
     int m = nc;
     unsigned long long base_mass = c_above, base_cnt = n_above;
+    double wk = 0.0, wd = 0.0;  // fp64 weights of the window's kept / dropped candidates
     const int nsub = (b2 - b1 + 1) * kSubPerBin;
     if (direct && nsub <= kSub) {
       for (int i = tid; i < nsub; i += kSelThreads) { S.sub_mass[i] = 0ull; S.sub_cnt[i] = 0u; }
@@ -543,12 +576,16 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
         // keys of the cut sub-bin to sort; keys of the sub-bins above are kept
         for (int i = tid; i < nc; i += kSelThreads) {
           const unsigned long long ck = S.mcand[i];
-          const int sb = sub_of(weight_arg(key_value((uint32_t)(ck >> 32)), M, s2));
+          const float a = weight_arg(key_value((uint32_t)(ck >> 32)), M, s2);
+          const int sb = sub_of(a);
           if (sb == sstar) {
             const unsigned int slot = atomicAdd(&S.ncand, 1u);
             S.cand[slot] = ck;
           } else if (sb < sstar) {
             atomicAdd(&cc[(0xffffffffu - (uint32_t)(ck & 0xffffffffull)) / chunk], 1u);
+            wk += (double)exp2f(-a);
+          } else {
+            wd += (double)exp2f(-a);
           }
         }
         __syncthreads();
@@ -587,13 +624,13 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
 
     constexpr int E = kCap / kSelThreads;  // consecutive sorted keys per thread
     unsigned long long wloc[E], wsum = 0ull;
+    float wfl[E];
 #pragma unroll
     for (int j = 0; j < E; ++j) {
       const int i = tid * E + j;
-      unsigned long long w = 0ull;
-      if (i < m) w = fixed_mass(weight(key_value((uint32_t)(srt[i] >> 32)), M, s2), two_s);
-      wloc[j] = w;
-      wsum += w;
+      wfl[j] = (i < m) ? weight(key_value((uint32_t)(srt[i] >> 32)), M, s2) : 0.0f;
+      wloc[j] = fixed_mass(wfl[j], two_s);
+      wsum += wloc[j];
     }
     unsigned long long tmp;
     unsigned long long cum = base_mass + block_scan_excl(wsum, &tmp, S);
@@ -614,6 +651,12 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       pos = m > 0 ? m - 1 : 0;  // srt[0] is the zero pad when m == 0
     }
     const unsigned long long thr = srt[pos];
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const int i = tid * E + j;
+      if (i <= pos) wk += (double)wfl[j]; else wd += (double)wfl[j];
+    }
+    block_sum2(wk, wd, S);
     if (direct) {  // kept keys of the sorted list, per chunk
       for (int i = tid; i <= pos && i < m; i += kSelThreads) {
         const uint32_t idx = 0xffffffffu - (uint32_t)(srt[i] & 0xffffffffull);
@@ -635,6 +678,16 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       r.Z = Z;
       r.C = C;
       r.tv = Z ? (double)(Z - C) / (double)Z : 0.0;
+      // kept = above the window + the window's kept candidates; dropped likewise
+      // (an oversized window recomputes both in the recount pass below)
+      double fa_row = 0.0, fb_row = 0.0;
+      for (int q = 0; q < CS; ++q) {
+        const SelShared* R = cluster.map_shared_rank(&S, q);
+        fa_row += R->fpart[0];
+        fb_row += R->fpart[1];
+      }
+      r.wh = fa_row + S.fsum[0];
+      r.wt = fb_row + S.fsum[1];
       sel[row] = r;
       k_out[row] = (int32_t)k;
       tv_out[row] = (float)r.tv;
@@ -646,15 +699,22 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   const uint32_t kstar = S0->res_kstar;
   const uint32_t istar = S0->res_istar;
   const unsigned long long k_total = S0->res_k;
-  if (!direct) {  // recount: kept keys per chunk from the threshold
+  if (!direct) {  // recount: kept keys per chunk, and both weight sums, from the threshold
+    double fk = 0.0, fd = 0.0;
     for_each_quad<4>(ur, lo, hi, vec, [&](const float* x, int64_t i, const bool* ok) {
       unsigned int kept = 0u;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        kept += (ok[e] && is_kept(order_key(x[e]), (uint32_t)(i + e), kstar, istar)) ? 1u : 0u;
+      for (int e = 0; e < 4; ++e) {
+        if (!ok[e]) continue;
+        const bool k = is_kept(order_key(x[e]), (uint32_t)(i + e), kstar, istar);
+        const double w = (double)weight(x[e], M, s2);
+        if (k) { ++kept; fk += w; } else { fd += w; }
+      }
       const unsigned int tot = __reduce_add_sync(0xffffffffu, kept);
       if (lane == 0 && tot) atomicAdd(&cc[(uint32_t)i / chunk], tot);
     });
+    block_sum2(fk, fd, S);
+    if (tid == 0) { S.fpart[0] = S.fsum[0]; S.fpart[1] = S.fsum[1]; }
     __syncthreads();
   }
   // exclusive scan over this CTA's chunks (in blocks of kSelThreads chunks)
@@ -671,6 +731,16 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
     o = warp_sum(o);
     if (lane == 0) S.offset = o;
   }
+  if (!direct && rank == 0 && tid == 0) {  // the recount's weight sums, in rank order
+    double fk = 0.0, fd = 0.0;
+    for (int q = 0; q < CS; ++q) {
+      const SelShared* R = cluster.map_shared_rank(&S, q);
+      fk += R->fpart[0];
+      fd += R->fpart[1];
+    }
+    sel[row].wh = fk;
+    sel[row].wt = fd;
+  }
   cluster.sync();  // no CTA reads another's shared memory after this point
   unsigned long long offset = S.offset;
   if (tid == 0 && rank == CS - 1 && offset + run != k_total) atomicOr(status, CTA_DEV_INTERNAL);
@@ -682,13 +752,43 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
     if (c < c1) cc[c] = (uint32_t)(offset + ex);
     offset += tot;
   }
+  __syncthreads();  // this CTA's chunk offsets are written
+
+  // ---- 6. the kept indices of this segment, ascending ------------------------
+  // One warp per chunk: a running position from the chunk's offset, 32 keys
+  // per ballot, kIdxBatch words of logits in flight (they are still in L2).
+  int32_t* dst = idx_out + row * n;
+  for (int c = c0 + warp; c < c1; c += kSelWarps) {
+    const int64_t k0 = (int64_t)c * chunk;
+    const int nkc = (int)min((int64_t)chunk, n - k0);
+    uint32_t pos = __ldcg(cc + c);
+    for (int w0 = 0; w0 < nkc; w0 += kWarp * kIdxBatch) {
+      float x[kIdxBatch];
+#pragma unroll
+      for (int b = 0; b < kIdxBatch; ++b) {
+        const int i = w0 + b * kWarp + lane;
+        x[b] = i < nkc ? __ldcg(ur + k0 + i) : 0.0f;
+      }
+#pragma unroll
+      for (int b = 0; b < kIdxBatch; ++b) {
+        const int i = w0 + b * kWarp + lane;
+        const bool kept = i < nkc && is_kept(order_key(x[b]), (uint32_t)(k0 + i), kstar, istar);
+        const uint32_t m = __ballot_sync(0xffffffffu, kept);
+        if (kept) {
+          const uint32_t at = pos + __popc(m & ((1u << lane) - 1u));
+          if (at < (uint32_t)n) dst[at] = (int32_t)(k0 + i);
+        }
+        pos += __popc(m);
+      }
+    }
+  }
 }
 
 }  // namespace
 
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
-                          float* tv_out, uint32_t* chunk_off, const Plan& p, uint32_t* status,
-                          cudaStream_t st) {
+                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, const Plan& p,
+                          uint32_t* status, cudaStream_t st) {
   const size_t smem = sizeof(SelShared);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -705,7 +805,8 @@ cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, p, status);
+  e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, idx_out, p,
+                         status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
