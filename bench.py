@@ -202,9 +202,10 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     stream = torch.cuda.current_stream(device)
     nq = q_steps.shape[0]
 
-    def step(t, events=None):
+    def step(t, events=None, with_err=True):
         cta.cta_certified_topk_attn(q_steps[t % nq], K, V, eps, out=out, k_out=k_out, idx_out=idx,
-                                    tv_out=tv, err_out=err, kl_out=kl, workspace=ws,
+                                    tv_out=tv, err_out=err if with_err else None,
+                                    kl_out=kl if with_err else None, workspace=ws,
                                     status_dev=status, stream=stream, phase_events=events)
 
     for t in range(args.warmup):
@@ -240,6 +241,26 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     phase = [p / args.steps for p in phase]
     seconds = max_over_ranks(ms / 1e3, dist, device)
     value = aggregate(rows, args.steps, world, seconds)
+
+    # the same step without the error term and KL (out, k, idx, tv only): the
+    # dropped rows' value sums are skipped, so the output pass does half the FMAs
+    ne_steps = max(1, min(args.steps, 2000))
+    for t in range(3):
+        step(t, with_err=False)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for t in range(ne_steps):
+        step(t, ctypes.cast(handles[t], ctypes.c_void_p), with_err=False)
+    s1.record(stream)
+    torch.cuda.synchronize(device)
+    ne_seconds = max_over_ranks(s0.elapsed_time(s1) / 1e3, dist, device)
+    ne_phase = [0.0] * 4
+    for s in ev[:ne_steps]:
+        for j in range(4):
+            ne_phase[j] += s[j].elapsed_time(s[j + 1])
+    ne_phase = [p / ne_steps for p in ne_phase]
 
     # end to end through the public call with host buffers: q in, results out
     host_q = q_steps.cpu().pin_memory()
@@ -282,6 +303,9 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     dom_bytes = nbytes.get(dom_name, 0)
     achieved = dom_bytes / (phase[dom] / 1e3) / 1e9 if dom_bytes else None
     step_gbs = nbytes["step"] / (seconds / args.steps) / 1e9
+    ne_dom = max(range(4), key=lambda j: ne_phase[j])
+    ne_bytes = nbytes.get(names[ne_dom], 0)
+    ne_achieved = ne_bytes / (ne_phase[ne_dom] / 1e3) / 1e9 if ne_bytes else None
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": seconds * 1e3 / args.steps,
@@ -309,6 +333,16 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "q copied in from pinned host memory, out/k/tv/err/kl copied back every "
                         "step; the KV cache is resident and idx stays on the device"},
+        "no_err": {
+            "value": aggregate(rows, ne_steps, world, ne_seconds), "unit": UNIT,
+            "steps": ne_steps, "ms_per_step": ne_seconds * 1e3 / ne_steps,
+            "phase_ms": dict(zip(names, [round(p, 5) for p in ne_phase])),
+            "roofline": {"bound": "hbm", "kernel": names[ne_dom], "achieved": ne_achieved,
+                         "peak": peak, "unit": "GB/s",
+                         "frac": ne_achieved / peak if ne_achieved else None,
+                         "algorithmic_bytes_per_launch": ne_bytes},
+            "note": "err_out and kl_out not requested; timed after the main region",
+        },
         "gpu_launches": 4 * args.steps,
         "k_over_n_mean": float(k_out.float().mean().item() / prob.n),
         "clocks": clocks.summary(),
@@ -421,7 +455,8 @@ def main(argv=None):
                                         "steps": max(100, args.steps // 4)})
             r2 = run_libcta(sub, rank, world, local_rank)
             res["secondary"] = {k: r2[k] for k in ("value", "ms_per_step", "config", "roofline",
-                                                   "step_roofline", "phase_ms", "k_over_n_mean")}
+                                                   "step_roofline", "phase_ms", "k_over_n_mean",
+                                                   "no_err")}
         if res is not None and world == 1 and not args.no_cpu_baseline:
             from certified_top_sparse_b200 import workloads as W
             prob = W.decode128k() if args.workload == "decode128k" else W.decode32k()
