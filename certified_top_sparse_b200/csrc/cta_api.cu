@@ -169,9 +169,15 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   void** ev = opts->phase_events;
 
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_score(opts->dtype, q, K, u, cmax, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+  if ((score_tc_applies(p, opts->dtype) ? launch_score_tc(q, K, u, p, status, st)
+                                         : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) !=
+      cudaSuccess)
+    return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, p, status, st) != cudaSuccess)
+  if ((select_short_applies(p)
+           ? launch_select_short(u, sel, k_out, tv_out, idx_out, p, status, st)
+           : launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, p, status, st)) !=
+      cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
   if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)

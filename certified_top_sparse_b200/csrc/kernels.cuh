@@ -22,6 +22,21 @@ cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_
                           float* tv_out, uint32_t* chunk_off, int32_t* idx_out, const Plan& p,
                           uint32_t* status, cudaStream_t st);
 
+// Phase 1 on tcgen05 for the all-query case (bf16, d in {64, 128}, rows of a
+// KV group a multiple of 128, n a multiple of 256 and <= kShortMaxN): writes
+// the logits only (the short-row selection takes the row maxima itself).
+bool score_tc_applies(const Plan& p, int dtype);
+cudaError_t launch_score_tc(const void* q, const void* K, float* u, const Plan& p,
+                            uint32_t* status, cudaStream_t st);
+
+// Phase 2 for short rows (n <= kShortMaxN): one warp per row; same outputs as
+// launch_select (chunk_off unused).
+constexpr int kShortMaxN = 1024;
+bool select_short_applies(const Plan& p);
+cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
+                                int32_t* idx_out, const Plan& p, uint32_t* status,
+                                cudaStream_t st);
+
 // Phase 3: per-(row, chunk range) weighted value sums of kept (and dropped)
 // keys.  gather_ctas_per_sm: the CTAs per SM its launch is planned for.
 int gather_ctas_per_sm(bool want_err);

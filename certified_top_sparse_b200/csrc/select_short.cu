@@ -1,0 +1,267 @@
+// Phase 2 for short rows (n <= 1024, e.g. all-query self-attention): one warp
+// per row, the row's logits in registers.
+//
+// Method ("A Mathematical Theory of Top-k Sparse Attention via Total Variation
+// Distance", arXiv 2512.07647, abstract): certified Top-k keeps the minimal
+// k_eps whose discarded softmax mass (Z - C_k) / Z is <= eps, keys ranked by
+// logit (descending; ties by the lower index).
+//
+// The same exact arithmetic as the cluster selection: every weight w = 2^-a
+// (see weight() in common.cuh) becomes a 64-bit fixed-point integer, so every
+// mass sum is exact.  Per row:
+//   1. M = the row maximum; Z and the masses and counts of 64 coarse bins
+//      floor(a) (intervals of the ranking), one shared-memory histogram per warp;
+//   2. a warp scan finds the coarse bin holding the cut; a second histogram of
+//      64 fine bins floor(64 a) inside it finds the fine bin holding the cut;
+//   3. the fine bin's keys are taken in descending composite order (logit,
+//      then lower index) by repeated warp maxima until the kept mass is
+//      certified: that key is the last kept one (K*, I*);
+//   4. the fp64 sums of the kept and dropped weights, and the kept indices,
+//      ascending, written with ballots of 32 keys.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace cta {
+
+namespace {
+
+constexpr int kShortWarps = 8;
+constexpr int kHist = 64;  // bins per histogram level
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+    v = y > v ? y : v;
+  }
+  return v;
+}
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+template <typename U>
+__device__ __forceinline__ U warp_incl_scan(U v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const U y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// The bin (of kHist, two per lane in order) whose inclusion first certifies
+// the kept mass, given the mass and count ranked above the histogram.  On
+// return *before / *nbefore are the mass and count ranked above that bin.
+__device__ __forceinline__ int cut_bin(const unsigned long long* mass, const unsigned int* cnt,
+                                       unsigned long long Z, double eps, int lane,
+                                       unsigned long long* before, unsigned long long* nbefore) {
+  const unsigned long long m0 = mass[2 * lane], m1 = mass[2 * lane + 1];
+  const unsigned long long c0 = cnt[2 * lane], c1 = cnt[2 * lane + 1];
+  const unsigned long long incl = warp_incl_scan<unsigned long long>(m0 + m1, lane);
+  const unsigned long long cincl = warp_incl_scan<unsigned long long>(c0 + c1, lane);
+  const unsigned long long excl = *before + incl - m0 - m1;
+  const unsigned long long cexcl = *nbefore + cincl - c0 - c1;
+  const bool h0 = certified(Z, excl + m0, eps);
+  const bool h1 = certified(Z, excl + m0 + m1, eps);
+  const unsigned b1 = __ballot_sync(0xffffffffu, h1);
+  const int L = b1 ? __ffs(b1) - 1 : 31;  // the last lane's bins always certify
+  const bool first = __shfl_sync(0xffffffffu, h0, L);
+  const unsigned long long ex = __shfl_sync(0xffffffffu, excl, L);
+  const unsigned long long cx = __shfl_sync(0xffffffffu, cexcl, L);
+  const unsigned long long mL0 = __shfl_sync(0xffffffffu, m0, L);
+  const unsigned long long cL0 = __shfl_sync(0xffffffffu, c0, L);
+  *before = first ? ex : ex + mL0;
+  *nbefore = first ? cx : cx + cL0;
+  return first ? 2 * L : 2 * L + 1;
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 2 : 1)
+select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
+                    int32_t* __restrict__ k_out, float* __restrict__ tv_out,
+                    int32_t* __restrict__ idx_out, Plan p, uint32_t* __restrict__ status) {
+  __shared__ unsigned long long smass[kShortWarps][kHist];
+  __shared__ unsigned int scnt[kShortWarps][kHist];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * kShortWarps + warp;
+  if (row >= p.rows) return;  // whole warps only; no block-wide barrier below
+  const int n = (int)p.n;
+  const float s2 = p.scale2, two_s = p.two_s;
+  const float* ur = u + row * p.ustride;
+  unsigned long long* hm = smass[warp];
+  unsigned int* hc = scnt[warp];
+
+  float x[NPL];
+  float mx = kNegInf;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const int i = j * kWarp + lane;
+    x[j] = i < n ? ur[i] : kNegInf;
+    mx = fmaxf(mx, x[j]);
+  }
+  const float M = warp_max_f(mx);
+  const bool finite = isfinite(M);
+
+  // ---- 1. Z and the coarse histogram --------------------------------------
+  hm[lane] = 0ull; hm[lane + 32] = 0ull; hc[lane] = 0u; hc[lane + 32] = 0u;
+  __syncwarp();
+  unsigned long long z = 0ull;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    if (j * kWarp + lane < n) {
+      const float a = weight_arg(x[j], M, s2);
+      const unsigned long long W = fixed_mass(exp2f(-a), two_s);
+      const int cb = (int)fminf(a, (float)(kHist - 1));  // a >= 0; NaN clamps too
+      z += W;
+      atomicAdd(&hm[cb], W);
+      atomicAdd(&hc[cb], 1u);
+    }
+  }
+  const unsigned long long Z = warp_sum_u64(z);
+  __syncwarp();
+
+  // ---- 2. the coarse, then the fine bin holding the cut ---------------------
+  unsigned long long before = 0ull, nbefore = 0ull;
+  int cbs = kHist - 1, fbs = kHist - 1;
+  if (finite && Z > 0ull) {
+    cbs = cut_bin(hm, hc, Z, p.eps, lane, &before, &nbefore);
+    __syncwarp();
+    hm[lane] = 0ull; hm[lane + 32] = 0ull; hc[lane] = 0u; hc[lane + 32] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      if (j * kWarp + lane < n) {
+        const float a = weight_arg(x[j], M, s2);
+        if ((int)fminf(a, (float)(kHist - 1)) == cbs) {
+          const int fb = min(max((int)(a * (float)kHist) - cbs * kHist, 0), kHist - 1);
+          atomicAdd(&hm[fb], fixed_mass(exp2f(-a), two_s));
+          atomicAdd(&hc[fb], 1u);
+        }
+      }
+    }
+    __syncwarp();
+    fbs = cut_bin(hm, hc, Z, p.eps, lane, &before, &nbefore);
+  }
+
+  // ---- 3. walk the cut fine bin in descending composite order ---------------
+  uint32_t inmask = 0u;  // bit j: key j * 32 + lane lies in the cut fine bin
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    if (j * kWarp + lane < n) {
+      const float a = weight_arg(x[j], M, s2);
+      if ((int)fminf(a, (float)(kHist - 1)) == cbs &&
+          min(max((int)(a * (float)kHist) - cbs * kHist, 0), kHist - 1) == fbs)
+        inmask |= 1u << j;
+    }
+  }
+  unsigned long long cum = before, kk = nbefore, last = ~0ull, K = 0ull;
+  bool done = !(finite && Z > 0ull);
+  for (int guard = 0; !done && guard < n; ++guard) {
+    unsigned long long best = 0ull;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+      if ((inmask >> j) & 1u) {
+        const unsigned long long ck = composite(order_key(x[j]), (uint32_t)(j * kWarp + lane));
+        if (ck < last && ck > best) best = ck;
+      }
+    }
+    best = warp_max_u64(best);
+    if (best == 0ull) break;  // no key left: cannot happen for finite rows
+    K = best;
+    last = best;
+    cum += fixed_mass(weight(key_value((uint32_t)(best >> 32)), M, s2), two_s);
+    ++kk;
+    done = certified(Z, cum, p.eps);
+  }
+
+  uint32_t kstar, istar;
+  if (done && K != 0ull) {
+    kstar = (uint32_t)(K >> 32);
+    istar = 0xffffffffu - (uint32_t)(K & 0xffffffffull);
+  } else {  // non-finite row: keep every key, flag it
+    if (lane == 0) atomicOr(status, CTA_DEV_NONFINITE);
+    kstar = 0u;
+    istar = 0xffffffffu;
+    kk = (unsigned long long)n;
+    cum = Z;
+  }
+
+  // ---- 4. weight sums and the kept indices ---------------------------------
+  double fh = 0.0, fd = 0.0;
+  int32_t* dst = idx_out + row * n;
+  uint32_t pos = 0u;
+#pragma unroll
+  for (int j = 0; j < NPL; ++j) {
+    const int i = j * kWarp + lane;
+    bool kept = false;
+    if (i < n) {
+      kept = is_kept(order_key(x[j]), (uint32_t)i, kstar, istar);
+      const double w = (double)weight(x[j], M, s2);
+      if (kept) fh += w; else fd += w;
+    }
+    const uint32_t m = __ballot_sync(0xffffffffu, kept);
+    if (kept) {
+      const uint32_t at = pos + __popc(m & ((1u << lane) - 1u));
+      if (at < (uint32_t)n) dst[at] = (int32_t)i;
+    }
+    pos += __popc(m);
+  }
+  fh = warp_sum_f64(fh);
+  fd = warp_sum_f64(fd);
+  if (lane == 0) {
+    if (pos != (uint32_t)kk) atomicOr(status, CTA_DEV_INTERNAL);
+    RowSel r;
+    r.M = M;
+    r.kstar = kstar;
+    r.istar = (int32_t)istar;
+    r.k = (int32_t)kk;
+    r.Z = Z;
+    r.C = cum;
+    r.tv = Z ? (double)(Z - cum) / (double)Z : 0.0;
+    r.wh = fh;
+    r.wt = fd;
+    sel[row] = r;
+    k_out[row] = (int32_t)kk;
+    tv_out[row] = (float)r.tv;
+  }
+}
+
+template <int NPL>
+cudaError_t launch_short_t(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
+                           int32_t* idx_out, const Plan& p, uint32_t* status, cudaStream_t st) {
+  const unsigned grid = (unsigned)((p.rows + kShortWarps - 1) / kShortWarps);
+  select_short_kernel<NPL><<<grid, kShortWarps * kWarp, 0, st>>>(u, sel, k_out, tv_out, idx_out, p,
+                                                                 status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool select_short_applies(const Plan& p) { return p.n <= (int64_t)kShortMaxN; }
+
+cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
+                                int32_t* idx_out, const Plan& p, uint32_t* status,
+                                cudaStream_t st) {
+  const int npl = (int)((p.n + kWarp - 1) / kWarp);
+  if (npl <= 1) return launch_short_t<1>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  if (npl <= 2) return launch_short_t<2>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  if (npl <= 4) return launch_short_t<4>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  if (npl <= 8) return launch_short_t<8>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  if (npl <= 16) return launch_short_t<16>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  if (npl <= 32) return launch_short_t<32>(u, sel, k_out, tv_out, idx_out, p, status, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace cta
