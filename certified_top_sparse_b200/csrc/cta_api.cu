@@ -154,6 +154,8 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (rc != CTA_OK) return rc;
   p.want_err = opts->err_out != nullptr;
   set_ranges(&p, gather_ctas_per_sm(p.want_err));
+  // all-query tiles on the tensor cores: logits and value sums per 128-row tile
+  const bool tc = score_tc_applies(p, opts->dtype);
   const Layout L = layout(p);
   if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
     return CTA_ERR_WORKSPACE;
@@ -169,9 +171,8 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   void** ev = opts->phase_events;
 
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
-  if ((score_tc_applies(p, opts->dtype) ? launch_score_tc(q, K, u, p, status, st)
-                                         : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) !=
-      cudaSuccess)
+  if ((tc ? launch_score_tc(q, K, u, p, status, st)
+          : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
   if ((select_short_applies(p)
@@ -180,12 +181,18 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
       cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)
-    return CTA_ERR_CUDA;
-  if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-  if (launch_finalize(opts->dtype, sel, acc, out, opts->err_out, opts->kl_out, p, status, st) !=
-      cudaSuccess)
-    return CTA_ERR_CUDA;
+  if (tc) {  // value sums and finalisation in one tensor-core pass
+    if (launch_pv_tc(V, u, sel, out, opts->err_out, opts->kl_out, p, status, st) != cudaSuccess)
+      return CTA_ERR_CUDA;
+    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+  } else {
+    if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)
+      return CTA_ERR_CUDA;
+    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (launch_finalize(opts->dtype, sel, acc, out, opts->err_out, opts->kl_out, p, status, st) !=
+        cudaSuccess)
+      return CTA_ERR_CUDA;
+  }
   if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;
   return CTA_OK;
 }

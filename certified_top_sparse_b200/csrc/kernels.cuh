@@ -29,6 +29,12 @@ bool score_tc_applies(const Plan& p, int dtype);
 cudaError_t launch_score_tc(const void* q, const void* K, float* u, const Plan& p,
                             uint32_t* status, cudaStream_t st);
 
+// Phases 3 and 4 on tcgen05 for the same all-query case (score_tc_applies):
+// value sums and the finalisation (out, err, KL) of 128-row tiles.
+cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, void* out,
+                         float* err_out, float* kl_out, const Plan& p, uint32_t* status,
+                         cudaStream_t st);
+
 // Phase 2 for short rows (n <= kShortMaxN): one warp per row; same outputs as
 // launch_select (chunk_off unused).
 constexpr int kShortMaxN = 1024;
