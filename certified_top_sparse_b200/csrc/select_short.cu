@@ -9,13 +9,14 @@
 // The same exact arithmetic as the cluster selection: every weight w = 2^-a
 // (see weight() in common.cuh) becomes a 64-bit fixed-point integer, so every
 // mass sum is exact.  Per row:
-//   1. M = the row maximum; Z and the masses and counts of 64 coarse bins
-//      floor(a) (intervals of the ranking), one shared-memory histogram per warp;
-//   2. a warp scan finds the coarse bin holding the cut; a second histogram of
-//      64 fine bins floor(64 a) inside it finds the fine bin holding the cut;
-//   3. the fine bin's keys are taken in descending composite order (logit,
-//      then lower index) by repeated warp maxima until the kept mass is
-//      certified: that key is the last kept one (K*, I*);
+//   1. M = the row maximum, Z, and per key its exponent a;
+//   2. three levels of 64-bin histograms (bins floor(a), floor(64 a),
+//      floor(4096 a): intervals of the ranking; counts and masses in shared
+//      memory with 32-bit atomics, four copies against contention), each followed by a
+//      warp scan that finds the bin holding the cut;
+//   3. that bin's keys (almost always one or two) are taken in descending
+//      composite order (logit, then lower index) by repeated warp maxima until
+//      the kept mass is certified: that key is the last kept one (K*, I*);
 //   4. the fp64 sums of the kept and dropped weights, and the kept indices,
 //      ascending, written with ballots of 32 keys.
 #include "common.cuh"
@@ -61,14 +62,54 @@ __device__ __forceinline__ U warp_incl_scan(U v, int lane) {
   return v;
 }
 
+constexpr int kCopies = 4;  // histogram copies (lane % 4) against atomic contention
+constexpr int kDigit = 21;  // masses are added as three 21-bit digits (32-bit atomics)
+
+// One warp's histogram: per bin and copy, a count and three mass digits
+// (copies of a bin in adjacent words, so they sit in different banks).  A
+// digit sum over at most 1024 keys stays below 2^31.
+struct Hist {
+  unsigned int cnt[kHist][kCopies];
+  unsigned int dig[3][kHist][kCopies];
+};
+
+__device__ __forceinline__ void hist_add(Hist& h, int bin, int cp, unsigned long long W) {
+  constexpr unsigned long long mask = (1ull << kDigit) - 1ull;
+  atomicAdd(&h.cnt[bin][cp], 1u);
+  atomicAdd(&h.dig[0][bin][cp], (unsigned int)(W & mask));
+  atomicAdd(&h.dig[1][bin][cp], (unsigned int)((W >> kDigit) & mask));
+  atomicAdd(&h.dig[2][bin][cp], (unsigned int)(W >> (2 * kDigit)));
+}
+
+__device__ __forceinline__ void hist_bin(const Hist& h, int bin, unsigned long long* mass,
+                                         unsigned long long* cnt) {
+  unsigned long long d0 = 0ull, d1 = 0ull, d2 = 0ull, c = 0ull;
+#pragma unroll
+  for (int k = 0; k < kCopies; ++k) {
+    c += h.cnt[bin][k];
+    d0 += h.dig[0][bin][k];
+    d1 += h.dig[1][bin][k];
+    d2 += h.dig[2][bin][k];
+  }
+  *mass = d0 + (d1 << kDigit) + (d2 << (2 * kDigit));
+  *cnt = c;
+}
+
+__device__ __forceinline__ void clear_hist(Hist& h, int lane) {
+  unsigned int* w = &h.cnt[0][0];
+  constexpr int words = (int)(sizeof(Hist) / sizeof(unsigned int));
+#pragma unroll
+  for (int i = lane; i < words; i += kWarp) w[i] = 0u;
+}
+
 // The bin (of kHist, two per lane in order) whose inclusion first certifies
 // the kept mass, given the mass and count ranked above the histogram.  On
 // return *before / *nbefore are the mass and count ranked above that bin.
-__device__ __forceinline__ int cut_bin(const unsigned long long* mass, const unsigned int* cnt,
-                                       unsigned long long Z, double eps, int lane,
+__device__ __forceinline__ int cut_bin(const Hist& h, unsigned long long Z, double eps, int lane,
                                        unsigned long long* before, unsigned long long* nbefore) {
-  const unsigned long long m0 = mass[2 * lane], m1 = mass[2 * lane + 1];
-  const unsigned long long c0 = cnt[2 * lane], c1 = cnt[2 * lane + 1];
+  unsigned long long m0, m1, c0, c1;
+  hist_bin(h, 2 * lane, &m0, &c0);
+  hist_bin(h, 2 * lane + 1, &m1, &c1);
   const unsigned long long incl = warp_incl_scan<unsigned long long>(m0 + m1, lane);
   const unsigned long long cincl = warp_incl_scan<unsigned long long>(c0 + c1, lane);
   const unsigned long long excl = *before + incl - m0 - m1;
@@ -87,21 +128,33 @@ __device__ __forceinline__ int cut_bin(const unsigned long long* mass, const uns
   return first ? 2 * L : 2 * L + 1;
 }
 
+// Bin of a at histogram level l (0: floor(a), 1: floor(64 a), 2: floor(4096 a)),
+// relative to the cut bins chosen at the previous levels; -1 when a lies
+// outside them.  Every level's bins are intervals of the ranking.
+__device__ __forceinline__ int level_bin(float a, int l, int b0, int b1) {
+  const int c0 = (int)fminf(a, (float)(kHist - 1));
+  if (l == 0) return c0;
+  if (c0 != b0) return -1;
+  const int c1 = min(max((int)(a * (float)kHist) - b0 * kHist, 0), kHist - 1);
+  if (l == 1) return c1;
+  if (c1 != b1) return -1;
+  return min(max((int)(a * (float)(kHist * kHist)) - (b0 * kHist + b1) * kHist, 0), kHist - 1);
+}
+
 template <int NPL>
 __global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 2 : 1)
 select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
                     int32_t* __restrict__ k_out, float* __restrict__ tv_out,
                     int32_t* __restrict__ idx_out, Plan p, uint32_t* __restrict__ status) {
-  __shared__ unsigned long long smass[kShortWarps][kHist];
-  __shared__ unsigned int scnt[kShortWarps][kHist];
+  __shared__ Hist hist[kShortWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kShortWarps + warp;
   if (row >= p.rows) return;  // whole warps only; no block-wide barrier below
   const int n = (int)p.n;
   const float s2 = p.scale2, two_s = p.two_s;
   const float* ur = u + row * p.ustride;
-  unsigned long long* hm = smass[warp];
-  unsigned int* hc = scnt[warp];
+  Hist& hw = hist[warp];
+  const int cp = lane & (kCopies - 1);
 
   float x[NPL];
   float mx = kNegInf;
@@ -113,59 +166,42 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
   }
   const float M = warp_max_f(mx);
   const bool finite = isfinite(M);
-
-  // ---- 1. Z and the coarse histogram --------------------------------------
-  hm[lane] = 0ull; hm[lane + 32] = 0ull; hc[lane] = 0u; hc[lane + 32] = 0u;
-  __syncwarp();
+  // exponents once per key; masses W = fixed_mass(2^-a) where needed
+  float av[NPL];
   unsigned long long z = 0ull;
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
-    if (j * kWarp + lane < n) {
-      const float a = weight_arg(x[j], M, s2);
-      const unsigned long long W = fixed_mass(exp2f(-a), two_s);
-      const int cb = (int)fminf(a, (float)(kHist - 1));  // a >= 0; NaN clamps too
-      z += W;
-      atomicAdd(&hm[cb], W);
-      atomicAdd(&hc[cb], 1u);
-    }
+    av[j] = weight_arg(x[j], M, s2);
+    if (j * kWarp + lane < n) z += fixed_mass(exp2f(-av[j]), two_s);
   }
   const unsigned long long Z = warp_sum_u64(z);
-  __syncwarp();
 
-  // ---- 2. the coarse, then the fine bin holding the cut ---------------------
+  // ---- 1-2. three histogram levels narrow the cut to one bin of 1/4096 ------
   unsigned long long before = 0ull, nbefore = 0ull;
-  int cbs = kHist - 1, fbs = kHist - 1;
+  int bl[3] = {kHist - 1, kHist - 1, kHist - 1};
   if (finite && Z > 0ull) {
-    cbs = cut_bin(hm, hc, Z, p.eps, lane, &before, &nbefore);
-    __syncwarp();
-    hm[lane] = 0ull; hm[lane + 32] = 0ull; hc[lane] = 0u; hc[lane + 32] = 0u;
-    __syncwarp();
+#pragma unroll 1
+    for (int l = 0; l < 3; ++l) {
+      clear_hist(hw, lane);
+      __syncwarp();
 #pragma unroll
-    for (int j = 0; j < NPL; ++j) {
-      if (j * kWarp + lane < n) {
-        const float a = weight_arg(x[j], M, s2);
-        if ((int)fminf(a, (float)(kHist - 1)) == cbs) {
-          const int fb = min(max((int)(a * (float)kHist) - cbs * kHist, 0), kHist - 1);
-          atomicAdd(&hm[fb], fixed_mass(exp2f(-a), two_s));
-          atomicAdd(&hc[fb], 1u);
+      for (int j = 0; j < NPL; ++j) {
+        if (j * kWarp + lane < n) {
+          const int bb = level_bin(av[j], l, bl[0], bl[1]);
+          if (bb >= 0) hist_add(hw, bb, cp, fixed_mass(exp2f(-av[j]), two_s));
         }
       }
+      __syncwarp();
+      bl[l] = cut_bin(hw, Z, p.eps, lane, &before, &nbefore);
+      __syncwarp();
     }
-    __syncwarp();
-    fbs = cut_bin(hm, hc, Z, p.eps, lane, &before, &nbefore);
   }
 
-  // ---- 3. walk the cut fine bin in descending composite order ---------------
-  uint32_t inmask = 0u;  // bit j: key j * 32 + lane lies in the cut fine bin
+  // ---- 3. walk the cut bin in descending composite order -------------------
+  uint32_t inmask = 0u;  // bit j: key j * 32 + lane lies in the cut bin
 #pragma unroll
-  for (int j = 0; j < NPL; ++j) {
-    if (j * kWarp + lane < n) {
-      const float a = weight_arg(x[j], M, s2);
-      if ((int)fminf(a, (float)(kHist - 1)) == cbs &&
-          min(max((int)(a * (float)kHist) - cbs * kHist, 0), kHist - 1) == fbs)
-        inmask |= 1u << j;
-    }
-  }
+  for (int j = 0; j < NPL; ++j)
+    if (j * kWarp + lane < n && level_bin(av[j], 2, bl[0], bl[1]) == bl[2]) inmask |= 1u << j;
   unsigned long long cum = before, kk = nbefore, last = ~0ull, K = 0ull;
   bool done = !(finite && Z > 0ull);
   for (int guard = 0; !done && guard < n; ++guard) {
@@ -181,7 +217,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     if (best == 0ull) break;  // no key left: cannot happen for finite rows
     K = best;
     last = best;
-    cum += fixed_mass(weight(key_value((uint32_t)(best >> 32)), M, s2), two_s);
+    cum += fixed_mass(exp2f(-weight_arg(key_value((uint32_t)(best >> 32)), M, s2)), two_s);
     ++kk;
     done = certified(Z, cum, p.eps);
   }
@@ -208,7 +244,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     bool kept = false;
     if (i < n) {
       kept = is_kept(order_key(x[j]), (uint32_t)i, kstar, istar);
-      const double w = (double)weight(x[j], M, s2);
+      const double w = (double)exp2f(-av[j]);
       if (kept) fh += w; else fd += w;
     }
     const uint32_t m = __ballot_sync(0xffffffffu, kept);
