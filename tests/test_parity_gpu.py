@@ -91,6 +91,46 @@ def test_bert_small_all_query():
     g, o, rep = check(prob, prob.eps, "bert small")
 
 
+def _all_query(n, d, heads, dtype, seed, scale=1.0, levels=None):
+    """Self-attention shaped problem (m = n, one KV head per query head)."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, heads, n, d)) * scale
+    K = rng.standard_normal((1, heads, n, d))
+    V = rng.standard_normal((1, heads, n, d))
+    if levels is not None:  # keys drawn from a few distinct rows: many exactly tied logits
+        K = K[:, :, rng.integers(0, levels, n), :]
+    t = lambda a: torch.from_numpy(a.astype(np.float32)).to(dtype)
+    return W.Problem("allq", t(q), t(K), t(V), 0.01, 1, heads, heads, n, n, d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("want_err", [True, False])
+def test_all_query_tensor_core_path(d, want_err):
+    """bf16, 128-row tiles, n a multiple of 256: tcgen05 logits and value sums."""
+    prob = _all_query(512, d, 2, torch.bfloat16, seed=d + int(want_err))
+    check(prob, prob.eps, f"all-query tcgen05 d={d} err={want_err}", want_err=want_err,
+          want_kl=want_err)
+
+
+@pytest.mark.parametrize("n,dtype", [(384, torch.bfloat16), (512, torch.float32),
+                                     (1024, torch.bfloat16), (96, torch.float32)])
+def test_all_query_cuda_core_paths(n, dtype):
+    """Short rows outside the tensor-core shapes: CUDA-core logits, warp-per-row selection."""
+    prob = _all_query(n, 64, 2, dtype, seed=n)
+    check(prob, prob.eps, f"all-query n={n} {dtype}")
+
+
+@pytest.mark.parametrize("levels", [1, 3])
+def test_short_rows_exact_ties(levels):
+    """Keys from 1 or 3 distinct rows: whole bins of tied logits, resolved by the
+    lower index (all-equal logits keep exactly ceil((1 - eps) n) keys)."""
+    prob = _all_query(512, 64, 1, torch.bfloat16, seed=7, levels=levels)
+    g, o, rep = check(prob, prob.eps, f"short rows ties levels={levels}")
+    assert rep["exact"] == prob.rows
+    if levels == 1:
+        assert np.all(g["k"].reshape(-1) == 507)
+
+
 def test_sweep_cell_small():
     prob = W.sweep_cell(n=4096, sigma=2.0, m=64)
     for eps in W.SWEEP_EPS:
