@@ -204,9 +204,9 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
 
     def step(t, events=None, with_err=True):
         cta.cta_certified_topk_attn(q_steps[t % nq], K, V, eps, out=out, k_out=k_out, idx_out=idx,
-                                    tv_out=tv, err_out=err if with_err else None,
-                                    kl_out=kl if with_err else None, workspace=ws,
-                                    status_dev=status, stream=stream, phase_events=events)
+                                    tv_out=tv, err_out=err, kl_out=kl, want_err=with_err,
+                                    want_kl=with_err, workspace=ws, status_dev=status,
+                                    stream=stream, phase_events=events)
 
     for t in range(args.warmup):
         step(t)
@@ -352,6 +352,87 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     return res if rank == 0 else None
 
 
+def measured_bf16_tflops() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def run_all_query(steps: int, warmup: int) -> dict:
+    """The BERT-shaped all-query workload (self-attention, m = n = 512, d = 64,
+    bf16, 8 x 12 heads): logits and value sums on tcgen05, warp-per-row
+    selection.  Query rows per second, per-phase times, the tensor kernels'
+    MMA rate and the selection kernel's HBM rate."""
+    import torch
+    import certified_top_sparse_b200 as cta
+    from certified_top_sparse_b200 import workloads as W
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    prob = W.bert()
+    q, K, V = prob.q.to(device), prob.K.to(device), prob.V.to(device)
+    rshape = (prob.batch, prob.n_heads, prob.m)
+    out = torch.empty_like(q)
+    k_out = torch.empty(rshape, dtype=torch.int32, device=device)
+    idx = torch.empty((*rshape, prob.n), dtype=torch.int32, device=device)
+    tv = torch.empty(rshape, dtype=torch.float32, device=device)
+    err = torch.empty(rshape, dtype=torch.float32, device=device)
+    kl = torch.empty(rshape, dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                            batch=prob.batch, m=prob.m),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for s in ev:
+        for e in s:
+            e.record(stream)
+    handles = [(ctypes.c_void_p * 5)(*[e.cuda_event for e in s]) for s in ev]
+    result = {}
+    for with_err in (True, False):
+        def step(events=None):
+            cta.cta_certified_topk_attn(q, K, V, prob.eps, out=out, k_out=k_out, idx_out=idx,
+                                        tv_out=tv, err_out=err, kl_out=kl, want_err=with_err,
+                                        want_kl=with_err, workspace=ws, status_dev=status,
+                                        stream=stream, phase_events=events)
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(device)
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for t in range(steps):
+            step(ctypes.cast(handles[t], ctypes.c_void_p))
+        stop.record(stream)
+        torch.cuda.synchronize(device)
+        assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
+        sec = start.elapsed_time(stop) / 1e3
+        ph = [sum(s[j].elapsed_time(s[j + 1]) for s in ev) / steps for j in range(4)]
+        rows, n, d = prob.rows, prob.n, prob.d
+        qk_flop = 2.0 * rows * n * d
+        pv_flop = 2.0 * rows * n * d * (4 if with_err else 2)  # hi/lo parts; head (and tail)
+        sel_bytes = 4.0 * rows * n + 4.0 * float(k_out.sum().item())
+        peak_tf, peak_kind = measured_bf16_tflops()
+        hbm, _ = measured_peaks()
+        result["err_on" if with_err else "err_off"] = {
+            "value": rows * steps / sec, "unit": "query-rows/s", "ms_per_step": sec * 1e3 / steps,
+            "phase_ms": {"logits_tcgen05": round(ph[0], 5), "select": round(ph[1], 5),
+                         "values_tcgen05_and_finalise": round(ph[2], 5)},
+            "tensor": {"qk_tflops": qk_flop / (ph[0] / 1e3) / 1e12,
+                       "pv_tflops": pv_flop / (ph[2] / 1e3) / 1e12,
+                       "peak_bf16_tflops": peak_tf, "peak_source": peak_kind},
+            "select_roofline": {"bound": "hbm", "achieved": sel_bytes / (ph[1] / 1e3) / 1e9,
+                                "peak": hbm, "unit": "GB/s",
+                                "frac": sel_bytes / (ph[1] / 1e3) / 1e9 / hbm,
+                                "algorithmic_bytes": sel_bytes},
+        }
+    result["config"] = {"workload": "bert all-query: batch 8, 12 heads, m = n = 512, d = 64, bf16, "
+                                    "heads 6-11 with planted keys, eps = 0.01",
+                        "steps": steps, "warmup": warmup, "k_over_n_mean":
+                            float(k_out.float().mean().item() / prob.n)}
+    return result
+
+
 # --------------------------------------------------------------------------
 # the oracle (CPU) as the reference arm and the cpu_baseline leg
 
@@ -441,6 +522,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--secondary", choices=("decode32k", "none"), default="decode32k",
                     help="also measure this workload (same method, fewer steps) and nest it")
+    ap.add_argument("--all-query", choices=("bert", "none"), default="bert",
+                    help="also measure the BERT-shaped all-query workload (tensor-core path)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -457,6 +540,8 @@ def main(argv=None):
             res["secondary"] = {k: r2[k] for k in ("value", "ms_per_step", "config", "roofline",
                                                    "step_roofline", "phase_ms", "k_over_n_mean",
                                                    "no_err")}
+        if res is not None and args.all_query != "none" and world == 1:
+            res["all_query"] = run_all_query(steps=max(20, args.steps // 40), warmup=args.warmup)
         if res is not None and world == 1 and not args.no_cpu_baseline:
             from certified_top_sparse_b200 import workloads as W
             prob = W.decode128k() if args.workload == "decode128k" else W.decode32k()
