@@ -41,6 +41,7 @@ class cta_opts(ctypes.Structure):
         ("kl_out", ctypes.c_void_p),
         ("status_dev", ctypes.c_void_p),
         ("phase_events", ctypes.c_void_p),
+        ("gap_out", ctypes.c_void_p),
     ]
 
 
@@ -107,7 +108,7 @@ def cta_version() -> int:
 
 
 def make_opts(*, batch=1, m=1, dtype=CTA_BF16, stream=None, workspace=None, err_out=None,
-              kl_out=None, status_dev=None, phase_events=None) -> cta_opts:
+              kl_out=None, status_dev=None, phase_events=None, gap_out=None) -> cta_opts:
     o = cta_opts()
     load().cta_opts_init(ctypes.byref(o))
     o.batch, o.m, o.dtype = int(batch), int(m), int(dtype)
@@ -119,6 +120,7 @@ def make_opts(*, batch=1, m=1, dtype=CTA_BF16, stream=None, workspace=None, err_
     o.kl_out = None if kl_out is None else kl_out.data_ptr()
     o.status_dev = None if status_dev is None else status_dev.data_ptr()
     o.phase_events = phase_events
+    o.gap_out = None if gap_out is None else gap_out.data_ptr()
     return o
 
 
@@ -144,13 +146,15 @@ def _shape(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor):
 
 def cta_certified_topk_attn(q, K, V, eps, *, out=None, k_out=None, idx_out=None, tv_out=None,
                             err_out=None, kl_out=None, want_err=True, want_kl=True,
-                            workspace=None, status_dev=None, stream=None, phase_events=None):
+                            gap_out=None, want_gap=False, workspace=None, status_dev=None,
+                            stream=None, phase_events=None):
     """Certified Top-k attention through libcta.
 
     Returns a dict of device tensors: ``out`` [batch, n_heads, m, d],
     ``k`` [batch, n_heads, m] int32, ``idx`` [batch, n_heads, m, n] int32
-    (entries [0, k) of each row are the kept keys, ascending), ``tv``, ``err``
-    and ``kl`` [batch, n_heads, m] fp32 (``err``/``kl`` None when not wanted).
+    (entries [0, k) of each row are the kept keys, ascending), ``tv``, ``err``,
+    ``kl`` and ``gap`` (the single-gap certificate) [batch, n_heads, m] fp32
+    (``err``/``kl``/``gap`` None when not wanted).
     """
     batch, n_heads, m, d, n_kv_heads, n = _shape(q, K, V)
     dev = q.device
@@ -163,6 +167,8 @@ def cta_certified_topk_attn(q, K, V, eps, *, out=None, k_out=None, idx_out=None,
         err_out = torch.empty(rows, dtype=torch.float32, device=dev)
     if want_kl and kl_out is None:
         kl_out = torch.empty(rows, dtype=torch.float32, device=dev)
+    if want_gap and gap_out is None:
+        gap_out = torch.empty(rows, dtype=torch.float32, device=dev)
     code = _dtype_code(q)
     if workspace is None:
         nbytes = cta_workspace_size(n, d, n_heads, n_kv_heads, batch=batch, m=m, dtype=code)
@@ -171,14 +177,16 @@ def cta_certified_topk_attn(q, K, V, eps, *, out=None, k_out=None, idx_out=None,
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     o = make_opts(batch=batch, m=m, dtype=code, stream=_stream_handle(stream), workspace=workspace,
                   err_out=err_out if want_err else None, kl_out=kl_out if want_kl else None,
-                  status_dev=status_dev, phase_events=phase_events)
+                  status_dev=status_dev, phase_events=phase_events,
+                  gap_out=gap_out if want_gap else None)
     rc = load().cta_certified_topk_attn(_ptr(q), _ptr(K), _ptr(V), n, d, n_heads, n_kv_heads,
                                         float(eps), _ptr(out), _ptr(k_out), _ptr(idx_out),
                                         _ptr(tv_out), ctypes.byref(o))
     if rc != CTA_OK:
         raise CtaError(rc, "cta_certified_topk_attn")
     return {"out": out, "k": k_out, "idx": idx_out, "tv": tv_out,
-            "err": err_out if want_err else None, "kl": kl_out if want_kl else None}
+            "err": err_out if want_err else None, "kl": kl_out if want_kl else None,
+            "gap": gap_out if want_gap else None}
 
 
 def cta_dense_attn(q, K, V, *, out=None, stream=None):

@@ -33,6 +33,7 @@ struct Plan {
   int sel_cluster;      // CTAs (a thread-block cluster) per row in the selection pass
   int nranges;          // output pass: chunk ranges per (KV group, row tile)
   int range_len;        // chunks per range
+  int gparts;           // partial maxima of the dropped logits per row (one per selection CTA)
 };
 
 // Per-row result of the selection pass.

@@ -30,7 +30,7 @@ int ceil_log2(int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t u, cmax, sel, choff, acc, status, total;
+  size_t u, cmax, sel, choff, acc, gmax, status, total;
 };
 
 // Output pass: each CTA owns a contiguous range of chunks of one (group, row
@@ -94,6 +94,7 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   while (cs < 8 && rows * cs * 2 <= 2 * 148 && n / (cs * 2) >= 4096) cs *= 2;
   p->sel_cluster = cs;
   set_ranges(p, 2);
+  p->gparts = (p->n <= (int64_t)kShortMaxN) ? 1 : p->sel_cluster;
   return CTA_OK;
 }
 
@@ -105,6 +106,7 @@ Layout layout(const Plan& p) {
   L.sel = off;    off = align256(off + sizeof(RowSel) * (size_t)p.rows);
   L.choff = off;  off = align256(off + sizeof(uint32_t) * (size_t)p.rows * p.nchunks);
   L.acc = off;    off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks * 2 * p.d);
+  L.gmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * kMaxGParts);
   L.status = off; off = align256(off + sizeof(uint32_t));
   L.total = off;
   return L;
@@ -166,6 +168,7 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   RowSel* sel = reinterpret_cast<RowSel*>(ws + L.sel);
   uint32_t* choff = reinterpret_cast<uint32_t*>(ws + L.choff);
   float* acc = reinterpret_cast<float*>(ws + L.acc);
+  float* gmax = reinterpret_cast<float*>(ws + L.gmax);
   uint32_t* status = opts->status_dev ? opts->status_dev : reinterpret_cast<uint32_t*>(ws + L.status);
   cudaStream_t st = static_cast<cudaStream_t>(opts->stream);
   void** ev = opts->phase_events;
@@ -176,21 +179,22 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
     return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
   if ((select_short_applies(p)
-           ? launch_select_short(u, sel, k_out, tv_out, idx_out, p, status, st)
-           : launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, p, status, st)) !=
+           ? launch_select_short(u, sel, k_out, tv_out, idx_out, gmax, p, status, st)
+           : launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, gmax, p, status, st)) !=
       cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
   if (tc) {  // value sums and finalisation in one tensor-core pass
-    if (launch_pv_tc(V, u, sel, out, opts->err_out, opts->kl_out, p, status, st) != cudaSuccess)
+    if (launch_pv_tc(V, u, sel, gmax, out, opts->err_out, opts->kl_out, opts->gap_out, p, status,
+                     st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
   } else {
     if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-    if (launch_finalize(opts->dtype, sel, acc, out, opts->err_out, opts->kl_out, p, status, st) !=
-        cudaSuccess)
+    if (launch_finalize(opts->dtype, sel, acc, gmax, out, opts->err_out, opts->kl_out, opts->gap_out,
+                        p, status, st) != cudaSuccess)
       return CTA_ERR_CUDA;
   }
   if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;

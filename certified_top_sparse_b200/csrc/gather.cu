@@ -16,8 +16,8 @@
 // a fixed order (fp64 across warps) into one partial per row and range.  The
 // weight sums (normalisers) and the kept indices come from selection.
 // Phase 4 (one CTA per row) adds the range partials in fixed order and forms
-// mu_head (the output), mu_tail, err = tau ||mu_tail - mu_head|| and
-// KL = log(sum_all w / sum_head w).
+// mu_head (the output), mu_tail, err = tau ||mu_tail - mu_head||,
+// KL = log(sum_all w / sum_head w) and the single-gap certificate.
 #include <algorithm>
 
 #include "common.cuh"
@@ -424,32 +424,46 @@ cudaError_t launch_gather_d(const void* V, const float* u, const RowSel* sel, fl
 
 constexpr int kFinThreads = 256;
 
+// Single-gap certificate: u_k the last kept logit, g the largest dropped one.
+__device__ __forceinline__ double single_gap_bound(double u_k, double g, int64_t k, int64_t n,
+                                                   int d) {
+  if (k >= n || !(g > -INFINITY)) return 0.0;
+  const double ratio = (double)k / (double)(n - k);
+  return 1.0 / (1.0 + ratio * exp((u_k - g) / sqrt((double)d)));
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kFinThreads)
 finalize_kernel(const RowSel* __restrict__ sel, const float* __restrict__ acc,
-                T* __restrict__ out, float* __restrict__ err_out, float* __restrict__ kl_out,
-                Plan p, uint32_t* __restrict__ status) {
+                const float* __restrict__ gmax, T* __restrict__ out, float* __restrict__ err_out,
+                float* __restrict__ kl_out, float* __restrict__ gap_out, Plan p,
+                uint32_t* __restrict__ status) {
   constexpr int G = kFinThreads / D;   // thread groups, each over every G-th chunk range
   __shared__ double s_ah[G][D], s_at[G][D];
   __shared__ double red[D / 32];
+  __shared__ float s_g[G];
   const int64_t row = blockIdx.x;
   const int dim = threadIdx.x % D;
   const int grp = threadIdx.x / D;
   double ah = 0.0, at = 0.0;
+  float g = kNegInf;
   const float* a = acc + row * p.nranges * 2 * D + dim;
 #pragma unroll 4
   for (int c = grp; c < p.nranges; c += G) {
     ah += a[(int64_t)c * 2 * D];
     if (p.want_err) at += a[(int64_t)c * 2 * D + D];
   }
+  if (dim == 0)  // the selection CTAs' largest dropped logits
+    for (int c = grp; c < p.gparts; c += G) g = fmaxf(g, gmax[row * kMaxGParts + c]);
   s_ah[grp][dim] = ah;
   s_at[grp][dim] = at;
+  if (dim == 0) s_g[grp] = g;
   __syncthreads();
   if (threadIdx.x >= D) return;
   ah = 0.0; at = 0.0;
-  for (int g = 0; g < G; ++g) {  // fixed order
-    ah += s_ah[g][dim];
-    at += s_at[g][dim];
+  for (int q = 0; q < G; ++q) {  // fixed order
+    ah += s_ah[q][dim];
+    at += s_at[q][dim];
   }
   const RowSel rs = sel[row];
   const double wh = rs.wh, wt = rs.wt;
@@ -470,17 +484,23 @@ finalize_kernel(const RowSel* __restrict__ sel, const float* __restrict__ acc,
     }
   }
   if (kl_out && dim == 0) kl_out[row] = (float)log1p(wt / wh);
+  if (gap_out && dim == 0) {
+    float gg = kNegInf;
+    for (int q = 0; q < G; ++q) gg = fmaxf(gg, s_g[q]);
+    gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gg, rs.k, p.n, D);
+  }
 }
 
 template <typename T>
-cudaError_t launch_finalize_t(const RowSel* sel, const float* acc, void* out, float* err_out,
-                              float* kl_out, const Plan& p, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_finalize_t(const RowSel* sel, const float* acc, const float* gmax, void* out,
+                              float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                              uint32_t* status, cudaStream_t st) {
   if (p.d == 64)
     finalize_kernel<T, 64><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
-        sel, acc, static_cast<T*>(out), err_out, kl_out, p, status);
+        sel, acc, gmax, static_cast<T*>(out), err_out, kl_out, gap_out, p, status);
   else
     finalize_kernel<T, 128><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
-        sel, acc, static_cast<T*>(out), err_out, kl_out, p, status);
+        sel, acc, gmax, static_cast<T*>(out), err_out, kl_out, gap_out, p, status);
   return cudaGetLastError();
 }
 
@@ -497,11 +517,13 @@ cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel
                    : launch_gather_d<__nv_bfloat16, 128>(V, u, sel, acc, p, status, st);
 }
 
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, void* out,
-                            float* err_out, float* kl_out, const Plan& p, uint32_t* status,
-                            cudaStream_t st) {
-  if (dtype == kDtypeF32) return launch_finalize_t<float>(sel, acc, out, err_out, kl_out, p, status, st);
-  return launch_finalize_t<__nv_bfloat16>(sel, acc, out, err_out, kl_out, p, status, st);
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const float* gmax,
+                            void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                            uint32_t* status, cudaStream_t st) {
+  if (dtype == kDtypeF32)
+    return launch_finalize_t<float>(sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st);
+  return launch_finalize_t<__nv_bfloat16>(sel, acc, gmax, out, err_out, kl_out, gap_out, p, status,
+                                          st);
 }
 
 }  // namespace cta

@@ -16,11 +16,13 @@ constexpr int kDtypeBF16 = CTA_BF16;
 cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, float* cmax,
                          const Plan& p, uint32_t* status, cudaStream_t st);
 
-// Phase 2: per-row certified selection; writes sel, k_out, tv_out and the
-// kept indices (idx_out), using chunk_off as its per-chunk offset scratch.
+// Phase 2: per-row certified selection; writes sel, k_out, tv_out, the kept
+// indices (idx_out) and per CTA the largest dropped logit (gmax[row][rank],
+// p.gparts per row), using chunk_off as its per-chunk offset scratch.
+constexpr int kMaxGParts = 8;
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
-                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, const Plan& p,
-                          uint32_t* status, cudaStream_t st);
+                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, float* gmax,
+                          const Plan& p, uint32_t* status, cudaStream_t st);
 
 // Phase 1 on tcgen05 for the all-query case (bf16, d in {64, 128}, rows of a
 // KV group a multiple of 128, n a multiple of 256 and <= kShortMaxN): writes
@@ -31,28 +33,28 @@ cudaError_t launch_score_tc(const void* q, const void* K, float* u, const Plan& 
 
 // Phases 3 and 4 on tcgen05 for the same all-query case (score_tc_applies):
 // value sums and the finalisation (out, err, KL) of 128-row tiles.
-cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, void* out,
-                         float* err_out, float* kl_out, const Plan& p, uint32_t* status,
-                         cudaStream_t st);
+cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, const float* gmax,
+                         void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                         uint32_t* status, cudaStream_t st);
 
 // Phase 2 for short rows (n <= kShortMaxN): one warp per row; same outputs as
 // launch_select (chunk_off unused).
 constexpr int kShortMaxN = 1024;
 bool select_short_applies(const Plan& p);
 cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                                int32_t* idx_out, const Plan& p, uint32_t* status,
+                                int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
                                 cudaStream_t st);
 
 // Phase 3: per-(row, chunk range) weighted value sums of kept (and dropped)
 // keys.  gather_ctas_per_sm: the CTAs per SM its launch is planned for.
 int gather_ctas_per_sm(bool want_err);
-cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel,
-                          float* acc, const Plan& p, uint32_t* status, cudaStream_t st);
+cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
+                          const Plan& p, uint32_t* status, cudaStream_t st);
 
 // Phase 4: combine chunk partials into out, err, kl.
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, void* out,
-                            float* err_out, float* kl_out, const Plan& p, uint32_t* status,
-                            cudaStream_t st);
+cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const float* gmax,
+                            void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                            uint32_t* status, cudaStream_t st);
 
 // Dense reference attention (all keys, fp32 online softmax).
 cudaError_t launch_dense(int dtype, const void* q, const void* K, const void* V, void* out,

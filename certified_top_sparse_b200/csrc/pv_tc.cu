@@ -16,7 +16,8 @@
 // O_head += (P_head,hi + P_head,lo) V and O_tail likewise in tensor memory;
 // A and V are double-buffered so the conversion of chunk j+1 overlaps the MMAs
 // of chunk j.  Each thread then finalises its row from tensor memory: out =
-// mu_head (fp64 division by selection's kept-weight sum), the error and KL.
+// mu_head (fp64 division by selection's kept-weight sum), the error, KL and
+// the single-gap certificate.
 #include <algorithm>
 
 #include "common.cuh"
@@ -110,8 +111,9 @@ struct PvSmem {
 template <int D, bool ERR>
 __global__ void __launch_bounds__(kPvThreads, 1)
 pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
-             const RowSel* __restrict__ sel, __nv_bfloat16* __restrict__ out,
-             float* __restrict__ err_out, float* __restrict__ kl_out, Plan p,
+             const RowSel* __restrict__ sel, const float* __restrict__ gmax,
+             __nv_bfloat16* __restrict__ out, float* __restrict__ err_out,
+             float* __restrict__ kl_out, float* __restrict__ gap_out, Plan p,
              uint32_t* __restrict__ status) {
   using S = PvSmem<D, ERR>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -265,6 +267,16 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
     if (!(wh > 0.0)) atomicOr(status, CTA_DEV_INTERNAL);
     if (err_out) err_out[row0 + r] = (float)(rs.C < rs.Z && wt > 0.0 ? rs.tv * sqrt(sq) : 0.0);
     if (kl_out) kl_out[row0 + r] = (float)log1p(wt / wh);
+    if (gap_out) {  // single-gap certificate from the last kept and the largest dropped logit
+      float g = kNegInf;
+      for (int c = 0; c < p.gparts; ++c) g = fmaxf(g, gmax[(row0 + r) * kMaxGParts + c]);
+      double b = 0.0;
+      if (rs.k < p.n && g > kNegInf) {
+        const double ratio = (double)rs.k / (double)(p.n - rs.k);
+        b = 1.0 / (1.0 + ratio * exp(((double)key_value(rs.kstar) - (double)g) / sqrt((double)D)));
+      }
+      gap_out[row0 + r] = (float)b;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -275,29 +287,34 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
 }
 
 template <int D, bool ERR>
-cudaError_t launch_pv_t(const void* V, const float* u, const RowSel* sel, void* out,
-                        float* err_out, float* kl_out, const Plan& p, uint32_t* status,
-                        cudaStream_t st) {
+cudaError_t launch_pv_t(const void* V, const float* u, const RowSel* sel, const float* gmax,
+                        void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                        uint32_t* status, cudaStream_t st) {
   const size_t smem = PvSmem<D, ERR>::kBytes;
   auto kern = pv_tc_kernel<D, ERR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(p.groups * (p.gm / kPvRows));
-  kern<<<grid, kPvThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(V), u, sel,
-                                       static_cast<__nv_bfloat16*>(out), err_out, kl_out, p, status);
+  kern<<<grid, kPvThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(V), u, sel, gmax,
+                                       static_cast<__nv_bfloat16*>(out), err_out, kl_out, gap_out,
+                                       p, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, void* out,
-                         float* err_out, float* kl_out, const Plan& p, uint32_t* status,
-                         cudaStream_t st) {
+cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, const float* gmax,
+                         void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                         uint32_t* status, cudaStream_t st) {
   if (p.d == 64)
-    return p.want_err ? launch_pv_t<64, true>(V, u, sel, out, err_out, kl_out, p, status, st)
-                      : launch_pv_t<64, false>(V, u, sel, out, err_out, kl_out, p, status, st);
-  return p.want_err ? launch_pv_t<128, true>(V, u, sel, out, err_out, kl_out, p, status, st)
-                    : launch_pv_t<128, false>(V, u, sel, out, err_out, kl_out, p, status, st);
+    return p.want_err ? launch_pv_t<64, true>(V, u, sel, gmax, out, err_out, kl_out, gap_out, p,
+                                              status, st)
+                      : launch_pv_t<64, false>(V, u, sel, gmax, out, err_out, kl_out, gap_out, p,
+                                               status, st);
+  return p.want_err ? launch_pv_t<128, true>(V, u, sel, gmax, out, err_out, kl_out, gap_out, p,
+                                             status, st)
+                    : launch_pv_t<128, false>(V, u, sel, gmax, out, err_out, kl_out, gap_out, p,
+                                              status, st);
 }
 
 }  // namespace cta

@@ -27,7 +27,8 @@
 //      of their exact masses gives the last kept key (K*, I*) and k_eps.
 //   5. Per output chunk, the exclusive offset of its first kept index.
 //   6. Each CTA writes the kept indices of its segment, ascending, from those
-//      offsets (one warp per chunk, ballots of 32 keys).
+//      offsets (one warp per chunk, ballots of 32 keys), and its segment's
+//      largest dropped logit (for the single-gap certificate).
 // Alongside, the fp64 sums of the kept and of the dropped weights (the output
 // normalisers): pass 3 sums the keys above and below the window, CTA 0 splits
 // the window's candidates at the cut; every reduction has a fixed order.
@@ -240,8 +241,8 @@ __device__ __forceinline__ unsigned long long bin_mass_lo(int b, int shift) {
 __global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSel* __restrict__ sel,
               int32_t* __restrict__ k_out, float* __restrict__ tv_out,
-              uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out, Plan p,
-              uint32_t* __restrict__ status) {
+              uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out,
+              float* __restrict__ gmax, Plan p, uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
@@ -758,6 +759,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   // One warp per chunk: a running position from the chunk's offset, 32 keys
   // per ballot, kIdxBatch words of logits in flight (they are still in L2).
   int32_t* dst = idx_out + row * n;
+  float dmax = kNegInf;  // the largest dropped logit of this CTA's segment
   for (int c = c0 + warp; c < c1; c += kSelWarps) {
     const int64_t k0 = (int64_t)c * chunk;
     const int nkc = (int)min((int64_t)chunk, n - k0);
@@ -773,6 +775,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       for (int b = 0; b < kIdxBatch; ++b) {
         const int i = w0 + b * kWarp + lane;
         const bool kept = i < nkc && is_kept(order_key(x[b]), (uint32_t)(k0 + i), kstar, istar);
+        if (i < nkc && !kept) dmax = fmaxf(dmax, x[b]);
         const uint32_t m = __ballot_sync(0xffffffffu, kept);
         if (kept) {
           const uint32_t at = pos + __popc(m & ((1u << lane) - 1u));
@@ -782,13 +785,15 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       }
     }
   }
+  dmax = block_max(dmax, S);
+  if (tid == 0) gmax[row * kMaxGParts + rank] = dmax;
 }
 
 }  // namespace
 
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
-                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, const Plan& p,
-                          uint32_t* status, cudaStream_t st) {
+                          float* tv_out, uint32_t* chunk_off, int32_t* idx_out, float* gmax,
+                          const Plan& p, uint32_t* status, cudaStream_t st) {
   const size_t smem = sizeof(SelShared);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -805,8 +810,8 @@ cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, idx_out, p,
-                         status);
+  e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, idx_out, gmax,
+                         p, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -17,8 +17,8 @@
 //   3. that bin's keys (almost always one or two) are taken in descending
 //      composite order (logit, then lower index) by repeated warp maxima until
 //      the kept mass is certified: that key is the last kept one (K*, I*);
-//   4. the fp64 sums of the kept and dropped weights, and the kept indices,
-//      ascending, written with ballots of 32 keys.
+//   4. the fp64 sums of the kept and dropped weights, the largest dropped
+//      logit, and the kept indices, ascending, written with ballots of 32 keys.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -145,7 +145,8 @@ template <int NPL>
 __global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 2 : 1)
 select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
                     int32_t* __restrict__ k_out, float* __restrict__ tv_out,
-                    int32_t* __restrict__ idx_out, Plan p, uint32_t* __restrict__ status) {
+                    int32_t* __restrict__ idx_out, float* __restrict__ gmax, Plan p,
+                    uint32_t* __restrict__ status) {
   __shared__ Hist hist[kShortWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kShortWarps + warp;
@@ -236,6 +237,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
 
   // ---- 4. weight sums and the kept indices ---------------------------------
   double fh = 0.0, fd = 0.0;
+  float dmax = kNegInf;  // the largest dropped logit
   int32_t* dst = idx_out + row * n;
   uint32_t pos = 0u;
 #pragma unroll
@@ -245,7 +247,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     if (i < n) {
       kept = is_kept(order_key(x[j]), (uint32_t)i, kstar, istar);
       const double w = (double)exp2f(-av[j]);
-      if (kept) fh += w; else fd += w;
+      if (kept) fh += w; else { fd += w; dmax = fmaxf(dmax, x[j]); }
     }
     const uint32_t m = __ballot_sync(0xffffffffu, kept);
     if (kept) {
@@ -256,6 +258,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
   }
   fh = warp_sum_f64(fh);
   fd = warp_sum_f64(fd);
+  dmax = warp_max_f(dmax);
   if (lane == 0) {
     if (pos != (uint32_t)kk) atomicOr(status, CTA_DEV_INTERNAL);
     RowSel r;
@@ -271,15 +274,17 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     sel[row] = r;
     k_out[row] = (int32_t)kk;
     tv_out[row] = (float)r.tv;
+    gmax[row * kMaxGParts] = dmax;
   }
 }
 
 template <int NPL>
 cudaError_t launch_short_t(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                           int32_t* idx_out, const Plan& p, uint32_t* status, cudaStream_t st) {
+                           int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
+                           cudaStream_t st) {
   const unsigned grid = (unsigned)((p.rows + kShortWarps - 1) / kShortWarps);
-  select_short_kernel<NPL><<<grid, kShortWarps * kWarp, 0, st>>>(u, sel, k_out, tv_out, idx_out, p,
-                                                                 status);
+  select_short_kernel<NPL><<<grid, kShortWarps * kWarp, 0, st>>>(u, sel, k_out, tv_out, idx_out,
+                                                                 gmax, p, status);
   return cudaGetLastError();
 }
 
@@ -288,15 +293,17 @@ cudaError_t launch_short_t(const float* u, RowSel* sel, int32_t* k_out, float* t
 bool select_short_applies(const Plan& p) { return p.n <= (int64_t)kShortMaxN; }
 
 cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                                int32_t* idx_out, const Plan& p, uint32_t* status,
+                                int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
                                 cudaStream_t st) {
   const int npl = (int)((p.n + kWarp - 1) / kWarp);
-  if (npl <= 1) return launch_short_t<1>(u, sel, k_out, tv_out, idx_out, p, status, st);
-  if (npl <= 2) return launch_short_t<2>(u, sel, k_out, tv_out, idx_out, p, status, st);
-  if (npl <= 4) return launch_short_t<4>(u, sel, k_out, tv_out, idx_out, p, status, st);
-  if (npl <= 8) return launch_short_t<8>(u, sel, k_out, tv_out, idx_out, p, status, st);
-  if (npl <= 16) return launch_short_t<16>(u, sel, k_out, tv_out, idx_out, p, status, st);
-  if (npl <= 32) return launch_short_t<32>(u, sel, k_out, tv_out, idx_out, p, status, st);
+#define CTA_SHORT(N) launch_short_t<N>(u, sel, k_out, tv_out, idx_out, gmax, p, status, st)
+  if (npl <= 1) return CTA_SHORT(1);
+  if (npl <= 2) return CTA_SHORT(2);
+  if (npl <= 4) return CTA_SHORT(4);
+  if (npl <= 8) return CTA_SHORT(8);
+  if (npl <= 16) return CTA_SHORT(16);
+  if (npl <= 32) return CTA_SHORT(32);
+#undef CTA_SHORT
   return cudaErrorInvalidValue;
 }
 

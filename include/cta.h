@@ -74,6 +74,15 @@ typedef struct {
   void** phase_events;    /* NULL, or 5 cudaEvent_t recorded on the stream before the score
                              phase, after it, after selection, after the output pass and
                              after finalisation (for timing individual phases)                */
+  float* gap_out;         /* [batch, n_heads, m] single-gap certificate, or NULL: with
+                             u_(k) the last kept and u_(k+1) the largest dropped logit,
+                             1 / (1 + k/(n-k) exp((u_(k) - u_(k+1)) / sqrt(d))), an upper
+                             bound on TV from the ordering alone (head logits >= u_(k), tail
+                             logits <= u_(k+1)); 0 when every key is kept.  The page "A
+                             Mathematical Theory of Top-k Sparse Attention via Total Variation
+                             Distance" (abstract) names deterministic bounds from ordered
+                             logits (single gap first) without printing them; this is the
+                             single-gap form derived from that ordering.                      */
 } cta_opts;
 
 /* Fill *o with the defaults listed above. */

@@ -24,6 +24,8 @@ Tolerances (the stated targets of the build, in writing):
 """
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import torch
 
@@ -145,6 +147,17 @@ def compare(prob: W.Problem, eps: float, gpu: dict, ora: dict, rows=None, window
         eo = ora["err"][ex]
         derr = np.abs(eg - eo)
         assert np.all(derr <= 1e-4 * eo + 1e-7), f"err off: max {derr.max()} (rel {np.max(derr / np.maximum(eo, 1e-30))})"
+    # single-gap certificate: the same gap up to the fp32 rounding of the two
+    # boundary logits (tie_bound covers both), and never below TV
+    if gpu.get("gap") is not None:
+        gg = gpu["gap"][rows].astype(np.float64)
+        assert np.all(gg >= gpu["tv"][rows].astype(np.float64) * (1 - 1e-6) - 1e-7), \
+            "single-gap bound below TV"
+        go = ora["gap_bound"][ex]
+        tb = np.nan_to_num(ora["tie_bound"][ex], nan=0.0)
+        tol = go * np.expm1(2.0 * tb / math.sqrt(prob.d)) + 1e-6 * go + 1e-9
+        dg = np.abs(gg[ex] - go)
+        assert np.all(dg <= tol), f"gap bound off: max {dg.max()} (tol {tol[np.argmax(dg)]})"
     return {
         "rows": nrow, "exact": int(exact.sum()), "differing_exempt": int((~exact).sum()),
         "classM": {f"{w:g}": int(classM[w].sum()) for w in WINDOWS}, "classT": int(classT.sum()),

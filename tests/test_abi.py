@@ -55,8 +55,9 @@ def test_version_and_strings():
 
 
 def test_opts_layout_matches_header():
-    # 4 int32, 3 pointers + size_t, 4 pointers on LP64
-    assert ctypes.sizeof(_lib.cta_opts) == 16 + 8 * 7
+    # 4 int32, 3 pointers + size_t, 5 pointers on LP64 (gap_out appended last)
+    assert ctypes.sizeof(_lib.cta_opts) == 16 + 8 * 8
+    assert _lib.cta_opts.gap_out.offset == 16 + 8 * 7
     o = _lib.make_opts()
     assert (o.batch, o.m, o.dtype) == (1, 1, cta.CTA_BF16)
 

@@ -33,6 +33,7 @@ def gpu_run(prob: W.Problem, eps: float, q=None, **kw):
     qq = (prob.q if q is None else q).to(dev)
     K, V = prob.K.to(dev), prob.V.to(dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    kw.setdefault("want_gap", True)
     res = cta.cta_certified_topk_attn(qq, K, V, eps, status_dev=status, **kw)
     torch.cuda.synchronize()
     h = to_host(res)
