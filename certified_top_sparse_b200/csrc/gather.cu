@@ -29,7 +29,7 @@ namespace {
 
 constexpr int kGWarps = 8;
 constexpr int kGatherThreads = kGWarps * kWarp;
-constexpr int kGStageBytes = 16384;
+constexpr int kGStageMax = 32768;  // bytes per V stage at most (128 keys of 256 B)
 
 template <typename T, int D, int RT>
 struct GatherCfg {
@@ -37,7 +37,8 @@ struct GatherCfg {
   static constexpr int LPK = ROWB / 16;             // lanes per key (16 bytes each)
   static constexpr int KPI = kWarp / LPK;           // keys per warp step
   static constexpr int NP = 16 / (int)sizeof(T) / 2;  // fp32 pairs per lane
-  static constexpr int TK = kGStageBytes / ROWB;    // keys per stage
+  static constexpr int TK = (kGStageMax / ROWB) < 128 ? kGStageMax / ROWB : 128;  // keys per stage
+  static constexpr int STAGE = TK * ROWB;           // bytes per stage
   static constexpr int STEPS = TK / (kGWarps * KPI);  // warp steps per stage
   static_assert(LPK >= 1 && LPK <= kWarp && kWarp % LPK == 0, "bad key width");
   static_assert(TK % (kGWarps * KPI) == 0, "a stage must split evenly over the warps");
@@ -107,7 +108,7 @@ struct GPieceIter {
 template <typename T, int D, int RT, bool ERR>
 struct GatherSmem {
   // dynamic bytes per CTA that let the planned number of CTAs share an SM
-  static constexpr size_t kBudget = ERR ? 110 * 1024 : 72 * 1024;
+  static constexpr size_t kBudget = 110 * 1024;
   using C = GatherCfg<T, D, RT>;
   static constexpr int KW = C::TK / kGWarps;          // keys per warp per stage
   static constexpr int WPK = RT * (ERR ? 2 : 1);      // (w, w) words per key: kept rows, dropped rows
@@ -116,9 +117,9 @@ struct GatherSmem {
   static constexpr size_t kW = sizeof(unsigned long long) * kGWarps * KW * WPK;  // per-warp weights
   static constexpr size_t kRed = sizeof(float) * kGWarps * 2 * D;  // item end; aliases kW
   static constexpr size_t kWR = kW > kRed ? kW : kRed;
-  static constexpr int kFit = (int)((kBudget - kWR) / kGStageBytes);
+  static constexpr int kFit = (int)((kBudget - kWR) / C::STAGE);
   static constexpr int kStages = kFit > 6 ? 6 : kFit;
-  static constexpr size_t kBytes = (size_t)kStages * kGStageBytes + kWR;
+  static constexpr size_t kBytes = (size_t)kStages * C::STAGE + kWR;
   static_assert(EPL <= 2, "at most two (key, row) pairs per lane");
   static_assert(kStages >= 3, "too few stages");
   static_assert(KW == C::KPI * C::STEPS, "warp keys per stage");
@@ -146,8 +147,9 @@ __device__ __forceinline__ void load_pairs(const unsigned long long* src, unsign
 // accumulators, and releases the stage; the last warp to release a fill
 // refills it.  The kernel is issue-bound, so the multiply-adds run without
 // branches (a dropped key multiplies a zero kept weight, and vice versa).
-// CTAs per SM: three without the error term (its registers allow it), two with.
-constexpr int gather_occupancy(bool err) { return err ? 2 : 3; }
+// CTAs per SM: two (32 KB stages; measured faster than three CTAs with 16 KB
+// stages even without the error term, whose registers would allow three).
+constexpr int gather_occupancy(bool) { return 2; }
 
 template <typename T, int D, int RT, bool ERR>
 __global__ void __launch_bounds__(kGatherThreads, gather_occupancy(ERR))
@@ -163,7 +165,7 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char* stage = smem_raw;                                         // [NS][16 KB]
-  unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem_raw + NS * kGStageBytes);
+  unsigned long long* wsm = reinterpret_cast<unsigned long long*>(smem_raw + NS * C::STAGE);
   float* red = reinterpret_cast<float*>(wsm);                              // [kGWarps][2][D]
   __shared__ unsigned long long full[NS];
   __shared__ int vcnt[NS];          // warps done with each stage (cumulative)
@@ -183,7 +185,7 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
     const unsigned char* src = reinterpret_cast<const unsigned char*>(
         V + ((int64_t)vprod.group * p.n + vprod.key0 + (int64_t)vprod.j * C::TK) * D);
     mbar_arrive_expect_tx(&full[s], bytes);
-    bulk_load(stage + s * kGStageBytes, src, bytes, &full[s], pol);
+    bulk_load(stage + s * C::STAGE, src, bytes, &full[s], pol);
     ++vissued;
     vprod.next(nitems, p);
   };
@@ -294,7 +296,7 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
           if (lane == 0) atomicOr(status, CTA_DEV_TIMEOUT);
           return;
         }
-        const uint4* stg = reinterpret_cast<const uint4*>(stage + s * kGStageBytes);
+        const uint4* stg = reinterpret_cast<const uint4*>(stage + s * C::STAGE);
 #pragma unroll
         for (int q = 0; q < C::STEPS; ++q) {
           const int e = q * C::KPI + slot;
