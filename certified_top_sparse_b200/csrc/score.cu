@@ -31,8 +31,8 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kScoreThreads = kWarps * kWarp;
-constexpr int kStageBytes = 16384;
-constexpr int kStages = 4;
+constexpr int kStageBytes = 32768;  // K rows per stage: 128 keys of 256 B
+constexpr int kStages = 2;
 
 template <typename T, int D, int RT>
 struct ScoreCfg {
@@ -43,7 +43,8 @@ struct ScoreCfg {
   static constexpr int TK = kStageBytes / ROWB;       // keys per stage
   static constexpr int NOUT = RT >= LPK ? RT / LPK : 1;  // rows each lane holds after the butterfly
   static_assert(LPK >= 1 && LPK <= kWarp && kWarp % LPK == 0, "bad key width");
-  static_assert(TK % (kWarps * KPI) == 0, "a stage must split evenly over the warps");
+  static_assert(TK % (2 * kWarps * KPI) == 0, "a stage must split into pairs of warp steps");
+  static constexpr int PAIRS = TK / (2 * kWarps * KPI);  // pairs of key steps per warp and stage
 };
 
 // Widen one 16-byte piece to EPC/2 packed fp32 pairs (64-bit registers).
@@ -106,24 +107,26 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
   constexpr int NP = C::EPC / 2;  // fp32 pairs per 16-byte piece
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  unsigned char* stage = smem_raw;                                        // [kStages][16 KB]
+  unsigned char* stage = smem_raw;                                        // [kStages][32 KB]
   float* su = reinterpret_cast<float*>(smem_raw + kStages * kStageBytes);  // [RT][su_stride]
   // Row stride of the staged logits: chunk + KPI puts the rows of one warp
   // step in different banks (chunk is a multiple of 256).
   const int su_stride = p.chunk + C::KPI;
-  __shared__ unsigned long long full[kStages], empty[kStages];
+  __shared__ unsigned long long full[kStages];
+  __shared__ int done_cnt[kStages];  // warps finished with each stage (cumulative)
   __shared__ float red[kWarps][RT];
+  // Copy issuer state: the last warp to release a stage refills it, so the
+  // state lives in shared memory.
+  __shared__ TileIter prod;
+  __shared__ int issued;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nitems = p.tiles_score * p.nchunks * p.groups;
   const unsigned long long pol = (p.tiles_score == 1) ? policy_evict_first() : policy_evict_last();
 
-  // Thread 0 issues the bulk copies, kStages tiles ahead of consumption: it
-  // refills a stage as soon as all warps have released it.
-  TileIter prod;
-  bool producing = true;
-  int issued = 0;
+  // Bulk copies run kStages tiles ahead of consumption; whichever warp is the
+  // last to release a stage issues its refill.
   auto issue_next = [&]() {
     if (!prod.valid(nitems)) return;
     const int s = issued % kStages;
@@ -139,9 +142,10 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kWarps);
+      done_cnt[s] = 0;
     }
     mbar_fence_init();
+    issued = 0;
     prod.start(blockIdx.x, nitems, p);
     for (int s = 0; s < kStages; ++s) issue_next();
   }
@@ -193,13 +197,16 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
       }
       const int nkt = min(C::TK, nk - j * C::TK);
       const uint4* st = reinterpret_cast<const uint4*>(stage + s * kStageBytes);
-      // Exactly two key steps per warp and stage: both dot products first, then
-      // both butterflies, so the two shuffle chains overlap.
-      static_assert(C::TK == 2 * kWarps * C::KPI, "two steps per warp and stage");
+      (void)ph;
+      // Pairs of key steps per warp: both dot products first, then both
+      // butterflies, so the two shuffle chains overlap.
+#pragma unroll
+      for (int hp = 0; hp < C::PAIRS; ++hp) {
+      const int kbase = hp * 2 * kWarps * C::KPI;
       float acc[2][RT];
 #pragma unroll
       for (int u2 = 0; u2 < 2; ++u2) {
-        const int key = warp * C::KPI + u2 * kWarps * C::KPI + slot;  // < TK
+        const int key = kbase + warp * C::KPI + u2 * kWarps * C::KPI + slot;  // < TK
         unsigned long long ka[NP], kb[NP];
         widen_pairs<T>(st[key * (C::ROWB / 16) + ca], ka);
         widen_pairs<T>(st[key * (C::ROWB / 16) + cb], kb);
@@ -217,7 +224,7 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
       XorReduce<RT, C::LPK / 2>::run(acc[1]);
 #pragma unroll
       for (int u2 = 0; u2 < 2; ++u2) {
-        const int key = warp * C::KPI + u2 * kWarps * C::KPI + slot;
+        const int key = kbase + warp * C::KPI + u2 * kWarps * C::KPI + slot;
         if (writer && key < nkt) {
 #pragma unroll
           for (int o = 0; o < C::NOUT; ++o) {
@@ -226,14 +233,19 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
           }
         }
       }
+      }  // pairs of key steps
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      if (threadIdx.x == 0 && producing && prod.valid(nitems)) {
-        // refill stage s with tile t + kStages once every warp has released it
-        if (mbar_wait(&empty[s], ph)) issue_next();
-        else { producing = false; atomicOr(status, CTA_DEV_TIMEOUT); }
+      if (lane == 0) {
+        // the last of the kWarps warps to release this fill refills it with
+        // tile t + kStages
+        __threadfence_block();
+        const int done = atomicAdd(&done_cnt[s], 1);
+        if (done == kWarps * (t / kStages) + kWarps - 1) {
+          __threadfence_block();
+          issue_next();
+          __threadfence_block();
+        }
       }
-      __syncwarp();
     }
 
     // item done: coalesced write-out, chunk maxima, non-finite check
