@@ -30,7 +30,7 @@ int ceil_log2(int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t u, cmax, sel, choff, acc, gmax, status, total;
+  size_t u, cmax, sel, choff, acc, gmax, unit, status, total;
 };
 
 // Output pass: each CTA owns a contiguous range of chunks of one (group, row
@@ -107,6 +107,7 @@ Layout layout(const Plan& p) {
   L.choff = off;  off = align256(off + sizeof(uint32_t) * (size_t)p.rows * p.nchunks);
   L.acc = off;    off = align256(off + sizeof(float) * (size_t)p.rows * p.nchunks * 2 * p.d);
   L.gmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * kMaxGParts);
+  L.unit = off;   off = align256(off + sizeof(uint32_t) * (size_t)p.rows);
   L.status = off; off = align256(off + sizeof(uint32_t));
   L.total = off;
   return L;
@@ -169,6 +170,7 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   uint32_t* choff = reinterpret_cast<uint32_t*>(ws + L.choff);
   float* acc = reinterpret_cast<float*>(ws + L.acc);
   float* gmax = reinterpret_cast<float*>(ws + L.gmax);
+  uint32_t* unit_cnt = reinterpret_cast<uint32_t*>(ws + L.unit);
   uint32_t* status = opts->status_dev ? opts->status_dev : reinterpret_cast<uint32_t*>(ws + L.status);
   cudaStream_t st = static_cast<cudaStream_t>(opts->stream);
   void** ev = opts->phase_events;
@@ -179,8 +181,9 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
     return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
   if ((select_short_applies(p)
-           ? launch_select_short(u, sel, k_out, tv_out, idx_out, gmax, p, status, st)
-           : launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, gmax, p, status, st)) !=
+           ? launch_select_short(u, sel, k_out, tv_out, idx_out, gmax, unit_cnt, p, status, st)
+           : launch_select(u, cmax, sel, k_out, tv_out, choff, idx_out, gmax, unit_cnt, p, status,
+                           st)) !=
       cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
@@ -189,13 +192,11 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
                      st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-  } else {
-    if (launch_gather(opts->dtype, V, u, sel, acc, p, status, st) != cudaSuccess)
+  } else {  // value sums, then the last CTA of each row tile finalises it
+    if (launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
+                      opts->kl_out, opts->gap_out, p, status, st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-    if (launch_finalize(opts->dtype, sel, acc, gmax, out, opts->err_out, opts->kl_out, opts->gap_out,
-                        p, status, st) != cudaSuccess)
-      return CTA_ERR_CUDA;
   }
   if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;
   return CTA_OK;

@@ -7,17 +7,19 @@
 // ||Attn - Attn_k||_2 = tau ||mu_tail - mu_head||_2.
 //
 // Phase 3: persistent CTAs, each owning a contiguous range of key chunks of
-// one (KV group, row tile).  Bulk copies (TMA) bring 16 KB stages of V rows
-// into shared memory.  Per stage every warp turns the logits of the keys it
-// will consume into weights, stored as duplicated fp32 pairs (kept, and with
-// the error wanted dropped, zero elsewhere) ready to be packed-FMA operands.
-// Each lane owns 16 bytes of a value row and accumulates w v as packed fp32
-// pairs across the whole range; at the range's end lanes and warps combine in
-// a fixed order (fp64 across warps) into one partial per row and range.  The
-// weight sums (normalisers) and the kept indices come from selection.
-// Phase 4 (one CTA per row) adds the range partials in fixed order and forms
-// mu_head (the output), mu_tail, err = tau ||mu_tail - mu_head||,
-// KL = log(sum_all w / sum_head w) and the single-gap certificate.
+// one (KV group, row tile).  Bulk copies (TMA) bring stages of up to 128 V
+// rows (32 KB) into shared memory.  Per stage every warp turns the logits of
+// the keys it will consume into weights, stored as duplicated fp32 pairs
+// (kept, and with the error wanted dropped, zero elsewhere) ready to be
+// packed-FMA operands.  Each lane owns 16 bytes of a value row and accumulates
+// w v as packed fp32 pairs across the whole range; at the range's end lanes
+// and warps combine in a fixed order (fp64 across warps) into one partial per
+// row and range.  The weight sums (normalisers), the kept indices and the
+// largest dropped logits come from selection.
+// Phase 4, in the same kernel: the last CTA to finish a (KV group, row tile)
+// adds its rows' range partials in a fixed order and forms mu_head (the
+// output), mu_tail, err = tau ||mu_tail - mu_head||, KL = log(sum_all w /
+// sum_head w) and the single-gap certificate.
 #include <algorithm>
 
 #include "common.cuh"
@@ -115,7 +117,10 @@ struct GatherSmem {
   static constexpr int NPAIR = KW * RT;               // (key, row) pairs per warp per stage
   static constexpr int EPL = (NPAIR + kWarp - 1) / kWarp;  // pairs per lane
   static constexpr size_t kW = sizeof(unsigned long long) * kGWarps * KW * WPK;  // per-warp weights
-  static constexpr size_t kRed = sizeof(float) * kGWarps * 2 * D;  // item end; aliases kW
+  // item end (aliases kW): per-warp fp32 partials, then the fp64 range sums
+  static constexpr size_t kRedF = sizeof(float) * kGWarps * 2 * D;
+  static constexpr size_t kRedD = sizeof(double) * RT * 2 * D;
+  static constexpr size_t kRed = kRedF > kRedD ? kRedF : kRedD;
   static constexpr size_t kWR = kW > kRed ? kW : kRed;
   static constexpr int kFit = (int)((kBudget - kWR) / C::STAGE);
   static constexpr int kStages = kFit > 6 ? 6 : kFit;
@@ -140,6 +145,14 @@ __device__ __forceinline__ void load_pairs(const unsigned long long* src, unsign
   }
 }
 
+// Single-gap certificate: u_k the last kept logit, g the largest dropped one.
+__device__ __forceinline__ double single_gap_bound(double u_k, double g, int64_t k, int64_t n,
+                                                   int d) {
+  if (k >= n || !(g > -INFINITY)) return 0.0;
+  const double ratio = (double)k / (double)(n - k);
+  return 1.0 / (1.0 + ratio * exp((u_k - g) / sqrt((double)d)));
+}
+
 // The CTA streams V through a ring of stages; no CTA barrier is taken until
 // the end of an item.  Each warp computes, per stage, the weights of exactly
 // the keys it will consume (one (key, row) pair per lane, logits prefetched a
@@ -154,7 +167,10 @@ constexpr int gather_occupancy(bool) { return 2; }
 template <typename T, int D, int RT, bool ERR>
 __global__ void __launch_bounds__(kGatherThreads, gather_occupancy(ERR))
 gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel* __restrict__ sel,
-              float* __restrict__ acc_out, Plan p, uint32_t* __restrict__ status) {
+              float* __restrict__ acc_out, uint32_t* __restrict__ unit_cnt,
+              const float* __restrict__ gmax, T* __restrict__ out, float* __restrict__ err_out,
+              float* __restrict__ kl_out, float* __restrict__ gap_out, Plan p,
+              uint32_t* __restrict__ status) {
   using C = GatherCfg<T, D, RT>;
   using S = GatherSmem<T, D, RT, ERR>;
   constexpr int NP = C::NP;
@@ -171,6 +187,8 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
   __shared__ int vcnt[NS];          // warps done with each stage (cumulative)
   __shared__ GPieceIter<C::TK> vprod;  // value-tile issuer state (whoever issues)
   __shared__ int vissued;
+  __shared__ int s_last;                 // this CTA finished the last range of its unit
+  __shared__ double s_wh[RT], s_wt[RT];  // the tile's rows' kept / dropped weight sums
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -382,11 +400,87 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
       }
       __syncthreads();
     }
+
+    // ---- the last CTA to finish a (KV group, row tile) finalises its rows ----
+    __threadfence();  // this CTA's partials, visible device-wide before the count
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t prev = atomicAdd(&unit_cnt[g.group * p.tiles_out + g.tile], 1u);
+      s_last = prev == (uint32_t)(p.nranges - 1);
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      if (threadIdx.x < nrows) {
+        s_wh[threadIdx.x] = sel[row0 + threadIdx.x].wh;
+        s_wt[threadIdx.x] = sel[row0 + threadIdx.x].wt;
+      }
+      // sums over the ranges, fixed order: one thread per (row, head/tail, 4 dims),
+      // 16-byte loads, eight in flight; fp64 sums staged in shared memory
+      double* fin = reinterpret_cast<double*>(red);  // [RT][2][D]
+      constexpr int NA = ERR ? 2 : 1;
+      for (int x = threadIdx.x; x < nrows * NA * (D / 4); x += kGatherThreads) {
+        const int r = x / (NA * (D / 4)), rem = x % (NA * (D / 4));
+        const int a = rem / (D / 4), d4 = rem % (D / 4);
+        const float4* src = reinterpret_cast<const float4*>(acc_out + (row0 + r) * p.nranges * 2 * D +
+                                                            a * D) + d4;
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll 8
+        for (int c = 0; c < p.nranges; ++c) {
+          const float4 v = __ldcg(src + (int64_t)c * (2 * D / 4));
+          s0 += (double)v.x; s1 += (double)v.y; s2 += (double)v.z; s3 += (double)v.w;
+        }
+        double* f = fin + (r * 2 + a) * D + 4 * d4;
+        f[0] = s0; f[1] = s1; f[2] = s2; f[3] = s3;
+      }
+      __syncthreads();
+      // every row of the tile at once: thread x -> (row x / D, dimension x % D)
+      for (int x = threadIdx.x; x < nrows * D; x += kGatherThreads) {
+        const int r = x / D, dim = x % D;
+        const double mu_h = fin[(r * 2 + 0) * D + dim] / s_wh[r];
+        Elem<T>::store1(out + (row0 + r) * D + dim, (float)mu_h);
+        if constexpr (ERR) {
+          const double diff = s_wt[r] > 0.0 ? fin[(r * 2 + 1) * D + dim] / s_wt[r] - mu_h : 0.0;
+          fin[(r * 2 + 1) * D + dim] = diff * diff;  // each element read and rewritten by one thread
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x < nrows) {  // thread r: row r's scalars
+        const int r = threadIdx.x;
+        const int64_t row = row0 + r;
+        const RowSel rs = sel[row];
+        const double wh = rs.wh, wt = rs.wt;
+        if (!(wh > 0.0)) atomicOr(status, CTA_DEV_INTERNAL);
+        if (err_out) {
+          double tot = 0.0;
+          for (int dim = 0; dim < D; ++dim) tot += fin[(r * 2 + 1) * D + dim];  // fixed order
+          err_out[row] = (float)(rs.C < rs.Z && wt > 0.0 ? rs.tv * sqrt(tot) : 0.0);
+        }
+        if (kl_out) kl_out[row] = (float)log1p(wt / wh);
+        if (gap_out) {
+          float gm = kNegInf;
+          for (int c = 0; c < p.gparts; ++c) gm = fmaxf(gm, __ldcg(gmax + row * kMaxGParts + c));
+          gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gm, rs.k, p.n,
+                                                 D);
+        }
+      }
+      __syncthreads();
+    }
   }
 }
 
+struct GatherOut {
+  float* acc;
+  uint32_t* unit_cnt;
+  const float* gmax;
+  void* out;
+  float* err_out;
+  float* kl_out;
+  float* gap_out;
+};
+
 template <typename T, int D, int RT, bool ERR>
-cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, float* acc,
+cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, const GatherOut& o,
                             const Plan& p, uint32_t* status, cudaStream_t st) {
   const size_t smem = GatherSmem<T, D, RT, ERR>::kBytes;
   auto kern = gather_kernel<T, D, RT, ERR>;
@@ -399,111 +493,28 @@ cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, fl
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long nitems = (long long)p.tiles_out * p.nranges * p.groups;
   const long long grid = std::min<long long>(nitems, (long long)std::max(per_sm, 1) * sms);
-  kern<<<(unsigned)grid, kGatherThreads, smem, st>>>(static_cast<const T*>(V), u, sel, acc, p,
-                                                     status);
+  kern<<<(unsigned)grid, kGatherThreads, smem, st>>>(
+      static_cast<const T*>(V), u, sel, o.acc, o.unit_cnt, o.gmax, static_cast<T*>(o.out),
+      o.err_out, o.kl_out, o.gap_out, p, status);
   return cudaGetLastError();
 }
 
 template <typename T, int D, bool ERR>
-cudaError_t launch_gather_e(const void* V, const float* u, const RowSel* sel, float* acc,
+cudaError_t launch_gather_e(const void* V, const float* u, const RowSel* sel, const GatherOut& o,
                             const Plan& p, uint32_t* status, cudaStream_t st) {
   switch (p.rt_out) {
-    case 1: return launch_gather_t<T, D, 1, ERR>(V, u, sel, acc, p, status, st);
-    case 2: return launch_gather_t<T, D, 2, ERR>(V, u, sel, acc, p, status, st);
-    case 4: return launch_gather_t<T, D, 4, ERR>(V, u, sel, acc, p, status, st);
+    case 1: return launch_gather_t<T, D, 1, ERR>(V, u, sel, o, p, status, st);
+    case 2: return launch_gather_t<T, D, 2, ERR>(V, u, sel, o, p, status, st);
+    case 4: return launch_gather_t<T, D, 4, ERR>(V, u, sel, o, p, status, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <typename T, int D>
-cudaError_t launch_gather_d(const void* V, const float* u, const RowSel* sel, float* acc,
+cudaError_t launch_gather_d(const void* V, const float* u, const RowSel* sel, const GatherOut& o,
                             const Plan& p, uint32_t* status, cudaStream_t st) {
-  return p.want_err ? launch_gather_e<T, D, true>(V, u, sel, acc, p, status, st)
-                    : launch_gather_e<T, D, false>(V, u, sel, acc, p, status, st);
-}
-
-// ---- phase 4 ------------------------------------------------------------------
-
-constexpr int kFinThreads = 256;
-
-// Single-gap certificate: u_k the last kept logit, g the largest dropped one.
-__device__ __forceinline__ double single_gap_bound(double u_k, double g, int64_t k, int64_t n,
-                                                   int d) {
-  if (k >= n || !(g > -INFINITY)) return 0.0;
-  const double ratio = (double)k / (double)(n - k);
-  return 1.0 / (1.0 + ratio * exp((u_k - g) / sqrt((double)d)));
-}
-
-template <typename T, int D>
-__global__ void __launch_bounds__(kFinThreads)
-finalize_kernel(const RowSel* __restrict__ sel, const float* __restrict__ acc,
-                const float* __restrict__ gmax, T* __restrict__ out, float* __restrict__ err_out,
-                float* __restrict__ kl_out, float* __restrict__ gap_out, Plan p,
-                uint32_t* __restrict__ status) {
-  constexpr int G = kFinThreads / D;   // thread groups, each over every G-th chunk range
-  __shared__ double s_ah[G][D], s_at[G][D];
-  __shared__ double red[D / 32];
-  __shared__ float s_g[G];
-  const int64_t row = blockIdx.x;
-  const int dim = threadIdx.x % D;
-  const int grp = threadIdx.x / D;
-  double ah = 0.0, at = 0.0;
-  float g = kNegInf;
-  const float* a = acc + row * p.nranges * 2 * D + dim;
-#pragma unroll 4
-  for (int c = grp; c < p.nranges; c += G) {
-    ah += a[(int64_t)c * 2 * D];
-    if (p.want_err) at += a[(int64_t)c * 2 * D + D];
-  }
-  if (dim == 0)  // the selection CTAs' largest dropped logits
-    for (int c = grp; c < p.gparts; c += G) g = fmaxf(g, gmax[row * kMaxGParts + c]);
-  s_ah[grp][dim] = ah;
-  s_at[grp][dim] = at;
-  if (dim == 0) s_g[grp] = g;
-  __syncthreads();
-  if (threadIdx.x >= D) return;
-  ah = 0.0; at = 0.0;
-  for (int q = 0; q < G; ++q) {  // fixed order
-    ah += s_ah[q][dim];
-    at += s_at[q][dim];
-  }
-  const RowSel rs = sel[row];
-  const double wh = rs.wh, wt = rs.wt;
-  const double mu_h = ah / wh;
-  Elem<T>::store1(out + row * D + dim, (float)mu_h);
-  if (!(wh > 0.0) && dim == 0) atomicOr(status, CTA_DEV_INTERNAL);
-  if (err_out) {
-    const double diff = (wt > 0.0) ? (at / wt - mu_h) : 0.0;
-    double s = diff * diff;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if ((dim & 31) == 0) red[dim >> 5] = s;
-    asm volatile("bar.sync 1, %0;" ::"r"(D));  // the first D threads only
-    if (dim == 0) {
-      double tot = 0.0;
-      for (int w = 0; w < D / 32; ++w) tot += red[w];
-      err_out[row] = (float)(rs.C < rs.Z && wt > 0.0 ? rs.tv * sqrt(tot) : 0.0);
-    }
-  }
-  if (kl_out && dim == 0) kl_out[row] = (float)log1p(wt / wh);
-  if (gap_out && dim == 0) {
-    float gg = kNegInf;
-    for (int q = 0; q < G; ++q) gg = fmaxf(gg, s_g[q]);
-    gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gg, rs.k, p.n, D);
-  }
-}
-
-template <typename T>
-cudaError_t launch_finalize_t(const RowSel* sel, const float* acc, const float* gmax, void* out,
-                              float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                              uint32_t* status, cudaStream_t st) {
-  if (p.d == 64)
-    finalize_kernel<T, 64><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
-        sel, acc, gmax, static_cast<T*>(out), err_out, kl_out, gap_out, p, status);
-  else
-    finalize_kernel<T, 128><<<(unsigned)p.rows, kFinThreads, 0, st>>>(
-        sel, acc, gmax, static_cast<T*>(out), err_out, kl_out, gap_out, p, status);
-  return cudaGetLastError();
+  return p.want_err ? launch_gather_e<T, D, true>(V, u, sel, o, p, status, st)
+                    : launch_gather_e<T, D, false>(V, u, sel, o, p, status, st);
 }
 
 }  // namespace
@@ -511,21 +522,15 @@ cudaError_t launch_finalize_t(const RowSel* sel, const float* acc, const float* 
 int gather_ctas_per_sm(bool want_err) { return gather_occupancy(want_err); }
 
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
-                          const Plan& p, uint32_t* status, cudaStream_t st) {
+                          uint32_t* unit_cnt, const float* gmax, void* out, float* err_out,
+                          float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
+                          cudaStream_t st) {
+  const GatherOut o{acc, unit_cnt, gmax, out, err_out, kl_out, gap_out};
   if (dtype == kDtypeF32)
-    return p.d == 64 ? launch_gather_d<float, 64>(V, u, sel, acc, p, status, st)
-                     : launch_gather_d<float, 128>(V, u, sel, acc, p, status, st);
-  return p.d == 64 ? launch_gather_d<__nv_bfloat16, 64>(V, u, sel, acc, p, status, st)
-                   : launch_gather_d<__nv_bfloat16, 128>(V, u, sel, acc, p, status, st);
-}
-
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const float* gmax,
-                            void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                            uint32_t* status, cudaStream_t st) {
-  if (dtype == kDtypeF32)
-    return launch_finalize_t<float>(sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st);
-  return launch_finalize_t<__nv_bfloat16>(sel, acc, gmax, out, err_out, kl_out, gap_out, p, status,
-                                          st);
+    return p.d == 64 ? launch_gather_d<float, 64>(V, u, sel, o, p, status, st)
+                     : launch_gather_d<float, 128>(V, u, sel, o, p, status, st);
+  return p.d == 64 ? launch_gather_d<__nv_bfloat16, 64>(V, u, sel, o, p, status, st)
+                   : launch_gather_d<__nv_bfloat16, 128>(V, u, sel, o, p, status, st);
 }
 
 }  // namespace cta

@@ -22,7 +22,7 @@ cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, floa
 constexpr int kMaxGParts = 8;
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
                           float* tv_out, uint32_t* chunk_off, int32_t* idx_out, float* gmax,
-                          const Plan& p, uint32_t* status, cudaStream_t st);
+                          uint32_t* unit_cnt, const Plan& p, uint32_t* status, cudaStream_t st);
 
 // Phase 1 on tcgen05 for the all-query case (bf16, d in {64, 128}, rows of a
 // KV group a multiple of 128, n a multiple of 256 and <= kShortMaxN): writes
@@ -42,19 +42,19 @@ cudaError_t launch_pv_tc(const void* V, const float* u, const RowSel* sel, const
 constexpr int kShortMaxN = 1024;
 bool select_short_applies(const Plan& p);
 cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                                int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
-                                cudaStream_t st);
+                                int32_t* idx_out, float* gmax, uint32_t* unit_cnt, const Plan& p,
+                                uint32_t* status, cudaStream_t st);
 
-// Phase 3: per-(row, chunk range) weighted value sums of kept (and dropped)
-// keys.  gather_ctas_per_sm: the CTAs per SM its launch is planned for.
+// Phases 3 and 4: per-(row, chunk range) weighted value sums of kept (and
+// dropped) keys, then (the last CTA of each (KV group, row tile), counted in
+// unit_cnt, which selection zeroes) out, err, KL and the single-gap bound.
+// gather_ctas_per_sm: the CTAs per SM its launch is planned for.
 int gather_ctas_per_sm(bool want_err);
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
-                          const Plan& p, uint32_t* status, cudaStream_t st);
+                          uint32_t* unit_cnt, const float* gmax, void* out, float* err_out,
+                          float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
+                          cudaStream_t st);
 
-// Phase 4: combine chunk partials into out, err, kl.
-cudaError_t launch_finalize(int dtype, const RowSel* sel, const float* acc, const float* gmax,
-                            void* out, float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                            uint32_t* status, cudaStream_t st);
 
 // Dense reference attention (all keys, fp32 online softmax).
 cudaError_t launch_dense(int dtype, const void* q, const void* K, const void* V, void* out,

@@ -242,7 +242,8 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSel* __restrict__ sel,
               int32_t* __restrict__ k_out, float* __restrict__ tv_out,
               uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out,
-              float* __restrict__ gmax, Plan p, uint32_t* __restrict__ status) {
+              float* __restrict__ gmax, uint32_t* __restrict__ unit_cnt, Plan p,
+              uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
@@ -267,6 +268,11 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   const bool vec = (n & 3) == 0;
   const float s2 = p.scale2, two_s = p.two_s;
   const uint32_t chunk = (uint32_t)p.chunk;
+
+  // The output pass counts finished ranges per (KV group, row tile): zeroed
+  // here by the tile's first row.
+  if (rank == 0 && tid == 0 && (row % p.gm) % p.rt_out == 0)
+    unit_cnt[(row / p.gm) * p.tiles_out + (row % p.gm) / p.rt_out] = 0u;
 
   // Row maximum from the per-chunk maxima of phase 1 (same in every CTA).
   float M = kNegInf;
@@ -793,7 +799,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
 
 cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_t* k_out,
                           float* tv_out, uint32_t* chunk_off, int32_t* idx_out, float* gmax,
-                          const Plan& p, uint32_t* status, cudaStream_t st) {
+                          uint32_t* unit_cnt, const Plan& p, uint32_t* status, cudaStream_t st) {
   const size_t smem = sizeof(SelShared);
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -811,7 +817,7 @@ cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, idx_out, gmax,
-                         p, status);
+                         unit_cnt, p, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -145,8 +145,8 @@ template <int NPL>
 __global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 2 : 1)
 select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
                     int32_t* __restrict__ k_out, float* __restrict__ tv_out,
-                    int32_t* __restrict__ idx_out, float* __restrict__ gmax, Plan p,
-                    uint32_t* __restrict__ status) {
+                    int32_t* __restrict__ idx_out, float* __restrict__ gmax,
+                    uint32_t* __restrict__ unit_cnt, Plan p, uint32_t* __restrict__ status) {
   __shared__ Hist hist[kShortWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kShortWarps + warp;
@@ -275,16 +275,19 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     k_out[row] = (int32_t)kk;
     tv_out[row] = (float)r.tv;
     gmax[row * kMaxGParts] = dmax;
+    // the output pass counts finished ranges per (KV group, row tile)
+    if ((row % p.gm) % p.rt_out == 0)
+      unit_cnt[(row / p.gm) * p.tiles_out + (row % p.gm) / p.rt_out] = 0u;
   }
 }
 
 template <int NPL>
 cudaError_t launch_short_t(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                           int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
-                           cudaStream_t st) {
+                           int32_t* idx_out, float* gmax, uint32_t* unit_cnt, const Plan& p,
+                           uint32_t* status, cudaStream_t st) {
   const unsigned grid = (unsigned)((p.rows + kShortWarps - 1) / kShortWarps);
   select_short_kernel<NPL><<<grid, kShortWarps * kWarp, 0, st>>>(u, sel, k_out, tv_out, idx_out,
-                                                                 gmax, p, status);
+                                                                 gmax, unit_cnt, p, status);
   return cudaGetLastError();
 }
 
@@ -293,10 +296,10 @@ cudaError_t launch_short_t(const float* u, RowSel* sel, int32_t* k_out, float* t
 bool select_short_applies(const Plan& p) { return p.n <= (int64_t)kShortMaxN; }
 
 cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, float* tv_out,
-                                int32_t* idx_out, float* gmax, const Plan& p, uint32_t* status,
-                                cudaStream_t st) {
+                                int32_t* idx_out, float* gmax, uint32_t* unit_cnt, const Plan& p,
+                                uint32_t* status, cudaStream_t st) {
   const int npl = (int)((p.n + kWarp - 1) / kWarp);
-#define CTA_SHORT(N) launch_short_t<N>(u, sel, k_out, tv_out, idx_out, gmax, p, status, st)
+#define CTA_SHORT(N) launch_short_t<N>(u, sel, k_out, tv_out, idx_out, gmax, unit_cnt, p, status, st)
   if (npl <= 1) return CTA_SHORT(1);
   if (npl <= 2) return CTA_SHORT(2);
   if (npl <= 4) return CTA_SHORT(4);
