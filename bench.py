@@ -343,7 +343,7 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
                          "algorithmic_bytes_per_launch": ne_bytes},
             "note": "err_out and kl_out not requested; timed after the main region",
         },
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 3 * args.steps,  # logits, selection, value sums + finalisation
         "k_over_n_mean": float(k_out.float().mean().item() / prob.n),
         "clocks": clocks.summary(),
     }
