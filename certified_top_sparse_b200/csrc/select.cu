@@ -53,7 +53,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kSubPerBin = 64;          // sub-bins per bin: 4096 per halving of the weight
 constexpr int kSub = 2048;              // sub-bins available (a window of up to 32 bins)
 constexpr int kLocalChunks = 1024;      // per-CTA chunk counters kept in shared memory
-constexpr int kIdxBatch = 8;            // 32-key words in flight per warp in the index pass
+constexpr int kIdxBatch = 16;           // 32-key words in flight per warp in the index pass
 constexpr int kBinsPerThread = kBins / kSelThreads;
 constexpr double kBoundSlack = 4e-6;    // covers exp2f's error (2 ulp) with margin
 constexpr double kDecideSlack = 1e-9;   // covers fp64 rounding in the exact test
@@ -73,6 +73,7 @@ struct SelShared {
   unsigned long long dmass[256];    // radix narrowing: digit masses (this CTA)
   unsigned int dcnt[256];           //                  digit counts (this CTA)
   unsigned long long warp_buf[kSelWarps];
+  unsigned long long warp_buf3[kSelWarps][3];
   double fwarp[kSelWarps][2];       // per-warp fp64 sums
   double fpart[2];                  // this CTA's fp64 weight sums: kept (above), dropped (below)
   double fsum[2];                   // block result of block_sum2
@@ -117,6 +118,46 @@ __device__ unsigned long long block_scan_excl(unsigned long long v, unsigned lon
   *total = S.warp_buf[kSelWarps - 1];
   __syncthreads();
   return before + x - v;
+}
+
+// Exclusive scans of three 64-bit values per thread at once (three barriers);
+// t[] gets the three block sums.
+__device__ void block_scan_excl3(unsigned long long* v, unsigned long long* t, SelShared& S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long x[3] = {v[0], v[1], v[2]};
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, x[k], o);
+      if (lane >= o) x[k] += y;
+    }
+  }
+  if (lane == 31) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) S.warp_buf3[warp][k] = x[k];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      unsigned long long w = (lane < kSelWarps) ? S.warp_buf3[lane][k] : 0ull;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < kSelWarps) S.warp_buf3[lane][k] = w;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const unsigned long long before = warp ? S.warp_buf3[warp - 1][k] : 0ull;
+    t[k] = S.warp_buf3[kSelWarps - 1][k];
+    v[k] = before + x[k] - v[k];
+  }
+  __syncthreads();
 }
 
 __device__ unsigned long long block_sum(unsigned long long v, SelShared& S) {
@@ -338,10 +379,10 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       hsum += hi_m[j];
       csum += cn[j];
     }
-    unsigned long long ZL, ZU, NN;
-    unsigned long long CL = block_scan_excl(lsum, &ZL, S);
-    unsigned long long CU = block_scan_excl(hsum, &ZU, S);
-    unsigned long long CN = block_scan_excl(csum, &NN, S);
+    unsigned long long sc[3] = {lsum, hsum, csum}, tot[3];
+    block_scan_excl3(sc, tot, S);
+    const unsigned long long ZL = tot[0], ZU = tot[1];
+    unsigned long long CL = sc[0], CU = sc[1], CN = sc[2];
     const double e_hi = p.eps * (1.0 - kDecideSlack), e_lo = p.eps * (1.0 + kDecideSlack);
     unsigned long long cn_before[kBinsPerThread];
 #pragma unroll
