@@ -109,7 +109,7 @@ struct PvSmem {
 };
 
 template <int D, bool ERR>
-__global__ void __launch_bounds__(kPvThreads, 1)
+__global__ void __launch_bounds__(kPvThreads, ERR ? 1 : 2)
 pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
              const RowSel* __restrict__ sel, const float* __restrict__ gmax,
              __nv_bfloat16* __restrict__ out, float* __restrict__ err_out,
@@ -152,6 +152,29 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
   const int nch = (int)(p.n / kPvKeys);
   bool ok = true;
 
+  // Chunk j + 1's logits and V pieces are loaded into registers while chunk j
+  // is converted and multiplied (software pipelining over the chunks).
+  constexpr int P = D / 8;                              // 16-byte pieces per V row
+  constexpr int VPT = kPvKeys * P / kPvThreads;         // V pieces per thread and chunk
+  static_assert(kPvKeys * P % kPvThreads == 0, "V pieces split evenly");
+  float x[32];
+  uint4 vv[VPT];
+  auto load_chunk = [&](int j, float* xs, uint4* vs) {
+    const float4* src = reinterpret_cast<const float4*>(ur + j * kPvKeys + half * 32);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float4 f = __ldg(src + e);
+      xs[4 * e] = f.x; xs[4 * e + 1] = f.y; xs[4 * e + 2] = f.z; xs[4 * e + 3] = f.w;
+    }
+    const __nv_bfloat16* vsrc = Vg + (int64_t)j * kPvKeys * D;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int q = threadIdx.x + i * kPvThreads, key = q / P, c = q % P;
+      vs[i] = __ldg(reinterpret_cast<const uint4*>(vsrc + (int64_t)key * D) + c);
+    }
+  };
+  if (nch > 0) load_chunk(0, x, vv);
+
   for (int j = 0; j < nch; ++j) {
     const int b = j & 1;
     // the MMAs that last read buffer b (chunk j - 2) must be done
@@ -159,15 +182,12 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
     if (__syncthreads_or(ok ? 0 : 1)) break;
     unsigned char* ab = abuf + b * S::kA;
     unsigned char* vb = vbuf + b * S::kV;
+    float xn[32];
+    uint4 vn[VPT];
+    if (j + 1 < nch) load_chunk(j + 1, xn, vn);
     // ---- weights of 32 keys of this row -> A operands (hi, lo; head, tail) --
     {
       const int k0 = j * kPvKeys + half * 32;
-      float x[32];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(ur + k0) + e);
-        x[4 * e] = f.x; x[4 * e + 1] = f.y; x[4 * e + 2] = f.z; x[4 * e + 3] = f.w;
-      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {  // 16-byte piece c of this thread's 64 bytes
         uint32_t hh[4], hl[4], th[4], tl[4];
@@ -196,14 +216,10 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
       }
     }
     // ---- the chunk's V rows (B operand, MN-major swizzled) -----------------
-    {
-      constexpr int P = D / 8;
-      const __nv_bfloat16* src = Vg + (int64_t)j * kPvKeys * D;
-      for (int x = threadIdx.x; x < kPvKeys * P; x += kPvThreads) {
-        const int key = x / P, c = x % P;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)key * D) + c);
-        *reinterpret_cast<uint4*>(vb + swz(key, c, kPvKeys)) = v;
-      }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int q = threadIdx.x + i * kPvThreads, key = q / P, c = q % P;
+      *reinterpret_cast<uint4*>(vb + swz(key, c, kPvKeys)) = vv[i];
     }
     fence_proxy_async();
     __syncthreads();
@@ -224,6 +240,10 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
       }
       tc_commit(&done[b]);
     }
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = xn[e];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) vv[i] = vn[i];
   }
   // ---- the last chunks' MMAs, then the sums out of tensor memory -----------
   if (ok && nch >= 1 && !mbar_wait(&done[(nch - 1) & 1], (unsigned)((nch - 1) >> 1) & 1u)) ok = false;
