@@ -7,12 +7,13 @@
 // the unscaled dot products u_i = q.k_i (the scale is folded into the weights).
 //
 // When every query of a head is a row (self-attention: m = n), QK^T is a dense
-// contraction, so it runs as tcgen05.mma (bf16 x bf16 -> fp32): one CTA of 128
+// contraction, so it runs as tcgen05.mma (bf16 x bf16 -> fp32): one CTA of 256
 // threads per (KV group, 128-row tile); Q (128 x d) and each 256-key chunk of K
 // (256 x d) are staged in shared memory in the 128-byte-swizzled K-major layout
 // the MMA descriptors describe; the 128 x 256 fp32 product accumulates in 256
-// tensor-memory columns; thread r reads row r (its TMEM lane) back with
-// tcgen05.ld and writes it to the logit buffer.  Exact products (bf16 x bf16
+// tensor-memory columns; each row (TMEM lane) is read back by two threads, one
+// per warpgroup and half of the columns, with tcgen05.ld and written to the
+// logit buffer.  Exact products (bf16 x bf16
 // fits fp32) accumulated in fp32, like the CUDA-core score kernel (the order
 // of the d-term sum differs).
 #include <algorithm>
@@ -26,7 +27,7 @@ namespace {
 
 constexpr int kTcRows = 128;     // M: query rows per CTA (one per thread and TMEM lane)
 constexpr int kTcN = 256;        // N: keys per MMA chunk (TMEM columns)
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;  // two warpgroups: same TMEM lanes (rows), half the columns each
 constexpr int kAtomRows = 8;     // rows per 128-byte swizzle atom
 constexpr int kRowBytes = 128;   // one atom row: 64 bf16 of K (the contraction dim)
 
@@ -114,6 +115,8 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   __shared__ uint32_t tmem_slot;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wg = warp >> 2;            // warpgroup: which half of the columns it reads back
+  const int rr = threadIdx.x & (kTcRows - 1);  // row (TMEM lane) of this thread
   const int tiles = p.gm / kTcRows;
   const int group = blockIdx.x / tiles, tile = blockIdx.x % tiles;
   const int64_t row0 = (int64_t)group * p.gm + (int64_t)tile * kTcRows;
@@ -132,9 +135,9 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const __nv_bfloat16* Kg = K + (int64_t)group * p.n * D;
-  float* urow = u + (row0 + threadIdx.x) * p.ustride;
+  float* urow = u + (row0 + rr) * p.ustride;
   constexpr uint32_t idesc = idesc_bf16_f32(kTcRows, kTcN);
   bool ok = true;
 
@@ -162,7 +165,7 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     if (ok) {
       tc_fence_after();
 #pragma unroll 1
-      for (int cb = 0; cb < kTcN / 32; ++cb) {
+      for (int cb = wg * (kTcN / 64); cb < (wg + 1) * (kTcN / 64); ++cb) {
         uint32_t v[32];
         tc_ld32(lane_addr + (uint32_t)(cb * 32), v);
         float4* dst = reinterpret_cast<float4*>(urow + (int64_t)c * kTcN + cb * 32);
