@@ -81,6 +81,7 @@ __device__ __forceinline__ void hist_add(Hist& h, int bin, int cp, unsigned long
   atomicAdd(&h.dig[2][bin][cp], (unsigned int)(W >> (2 * kDigit)));
 }
 
+
 __device__ __forceinline__ void hist_bin(const Hist& h, int bin, unsigned long long* mass,
                                          unsigned long long* cnt) {
   unsigned long long d0 = 0ull, d1 = 0ull, d2 = 0ull, c = 0ull;
@@ -128,21 +129,10 @@ __device__ __forceinline__ int cut_bin(const Hist& h, unsigned long long Z, doub
   return first ? 2 * L : 2 * L + 1;
 }
 
-// Bin of a at histogram level l (0: floor(a), 1: floor(64 a), 2: floor(4096 a)),
-// relative to the cut bins chosen at the previous levels; -1 when a lies
-// outside them.  Every level's bins are intervals of the ranking.
-__device__ __forceinline__ int level_bin(float a, int l, int b0, int b1) {
-  const int c0 = (int)fminf(a, (float)(kHist - 1));
-  if (l == 0) return c0;
-  if (c0 != b0) return -1;
-  const int c1 = min(max((int)(a * (float)kHist) - b0 * kHist, 0), kHist - 1);
-  if (l == 1) return c1;
-  if (c1 != b1) return -1;
-  return min(max((int)(a * (float)(kHist * kHist)) - (b0 * kHist + b1) * kHist, 0), kHist - 1);
-}
-
+// Latency-bound (a serial chain of scans and shuffles per row): as many rows
+// in flight as registers allow, four CTAs per SM up to 16 keys per lane.
 template <int NPL>
-__global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 2 : 1)
+__global__ void __launch_bounds__(kShortWarps * kWarp, NPL <= 16 ? 4 : 1)
 select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
                     int32_t* __restrict__ k_out, float* __restrict__ tv_out,
                     int32_t* __restrict__ idx_out, float* __restrict__ gmax,
@@ -167,42 +157,64 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
   }
   const float M = warp_max_f(mx);
   const bool finite = isfinite(M);
-  // exponents once per key; masses W = fixed_mass(2^-a) where needed
-  float av[NPL];
+  // the coarse histogram and Z in one loop (exponents recomputed where needed:
+  // cheaper than holding them in registers)
+  auto av = [&](int j) { return weight_arg(x[j], M, s2); };
+  uint32_t live = 0u;  // bit j: key j * 32 + lane exists (later: lies in the current cut bin)
+  clear_hist(hw, lane);
+  __syncwarp();
   unsigned long long z = 0ull;
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
-    av[j] = weight_arg(x[j], M, s2);
-    if (j * kWarp + lane < n) z += fixed_mass(exp2f(-av[j]), two_s);
+    if (j * kWarp + lane < n) {
+      live |= 1u << j;
+      const float a = av(j);
+      const unsigned long long W = fixed_mass(exp2f(-a), two_s);
+      z += W;
+      hist_add(hw, (int)fminf(a, (float)(kHist - 1)), cp, W);  // a >= 0; NaN clamps too
+    }
   }
   const unsigned long long Z = warp_sum_u64(z);
+  __syncwarp();
 
   // ---- 1-2. three histogram levels narrow the cut to one bin of 1/4096 ------
   unsigned long long before = 0ull, nbefore = 0ull;
-  int bl[3] = {kHist - 1, kHist - 1, kHist - 1};
   if (finite && Z > 0ull) {
+    const int b0 = cut_bin(hw, Z, p.eps, lane, &before, &nbefore);
+    uint32_t in = 0u;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+      if (((live >> j) & 1u) && (int)fminf(av(j), (float)(kHist - 1)) == b0) in |= 1u << j;
+    live = in;
+    // finer levels over the keys of the cut bin only: floor(64 a), floor(4096 a)
+    int base = b0;
 #pragma unroll 1
-    for (int l = 0; l < 3; ++l) {
+    for (int l = 1; l < 3; ++l) {
+      const float scale = l == 1 ? (float)kHist : (float)(kHist * kHist);
+      __syncwarp();
       clear_hist(hw, lane);
       __syncwarp();
 #pragma unroll
-      for (int j = 0; j < NPL; ++j) {
-        if (j * kWarp + lane < n) {
-          const int bb = level_bin(av[j], l, bl[0], bl[1]);
-          if (bb >= 0) hist_add(hw, bb, cp, fixed_mass(exp2f(-av[j]), two_s));
+      for (int j = 0; j < NPL; ++j)
+        if ((live >> j) & 1u) {
+          const float a = av(j);
+          const int bb = min(max((int)(a * scale) - base * kHist, 0), kHist - 1);
+          hist_add(hw, bb, cp, fixed_mass(exp2f(-a), two_s));
         }
-      }
       __syncwarp();
-      bl[l] = cut_bin(hw, Z, p.eps, lane, &before, &nbefore);
-      __syncwarp();
+      const int bl = cut_bin(hw, Z, p.eps, lane, &before, &nbefore);
+      in = 0u;
+#pragma unroll
+      for (int j = 0; j < NPL; ++j)
+        if (((live >> j) & 1u) && min(max((int)(av(j) * scale) - base * kHist, 0), kHist - 1) == bl)
+          in |= 1u << j;
+      live = in;
+      base = base * kHist + bl;
     }
   }
 
   // ---- 3. walk the cut bin in descending composite order -------------------
-  uint32_t inmask = 0u;  // bit j: key j * 32 + lane lies in the cut bin
-#pragma unroll
-  for (int j = 0; j < NPL; ++j)
-    if (j * kWarp + lane < n && level_bin(av[j], 2, bl[0], bl[1]) == bl[2]) inmask |= 1u << j;
+  const uint32_t inmask = live;  // bit j: key j * 32 + lane lies in the cut bin
   unsigned long long cum = before, kk = nbefore, last = ~0ull, K = 0ull;
   bool done = !(finite && Z > 0ull);
   for (int guard = 0; !done && guard < n; ++guard) {
@@ -246,7 +258,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
     bool kept = false;
     if (i < n) {
       kept = is_kept(order_key(x[j]), (uint32_t)i, kstar, istar);
-      const double w = (double)exp2f(-av[j]);
+      const double w = (double)exp2f(-av(j));
       if (kept) fh += w; else { fd += w; dmax = fmaxf(dmax, x[j]); }
     }
     const uint32_t m = __ballot_sync(0xffffffffu, kept);
