@@ -343,7 +343,9 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
                          "algorithmic_bytes_per_launch": ne_bytes},
             "note": "err_out and kl_out not requested; timed after the main region",
         },
-        "gpu_launches": 3 * args.steps,  # logits, selection, value sums + finalisation
+        # logits, selection, value sums, and (bf16 values with d = 128: the
+        # tensor-core value pass) a separate row-parallel finalisation kernel
+        "gpu_launches": (4 if (prob.V.dtype == torch.bfloat16 and prob.d == 128) else 3) * args.steps,
         "k_over_n_mean": float(k_out.float().mean().item() / prob.n),
         "clocks": clocks.summary(),
     }

@@ -34,6 +34,7 @@ struct Plan {
   int nranges;          // output pass: chunk ranges per (KV group, row tile)
   int range_len;        // chunks per range
   int gparts;           // partial maxima of the dropped logits per row (one per selection CTA)
+  int rstages;          // tensor-core output pass: 128-key stages per range (0: not used)
 };
 
 // Per-row result of the selection pass.

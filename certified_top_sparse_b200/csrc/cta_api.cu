@@ -115,6 +115,12 @@ Layout layout(const Plan& p) {
 
 bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
 
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
 int record(void** ev, int i, cudaStream_t st) {
   if (!ev) return CTA_OK;
   return cudaEventRecord((cudaEvent_t)ev[i], st) == cudaSuccess ? CTA_OK : CTA_ERR_CUDA;
@@ -159,6 +165,9 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   set_ranges(&p, gather_ctas_per_sm(p.want_err));
   // all-query tiles on the tensor cores: logits and value sums per 128-row tile
   const bool tc = score_tc_applies(p, opts->dtype);
+  // decode-shaped bf16 value sums on the tensor cores
+  const bool gtc = !tc && gather_tc_applies(p, opts->dtype);
+  if (gtc) set_ranges_tc(&p, sm_count());
   const Layout L = layout(p);
   if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
     return CTA_ERR_WORKSPACE;
@@ -193,8 +202,10 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
   } else {  // value sums, then the last CTA of each row tile finalises it
-    if (launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
-                      opts->kl_out, opts->gap_out, p, status, st) != cudaSuccess)
+    if ((gtc ? launch_gather_tc(V, u, sel, acc, gmax, out, opts->err_out, opts->kl_out,
+                                opts->gap_out, p, status, st)
+             : launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
+                             opts->kl_out, opts->gap_out, p, status, st)) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
   }

@@ -23,6 +23,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "finalize.cuh"
 #include "kernels.cuh"
 
 namespace cta {
@@ -143,14 +144,6 @@ __device__ __forceinline__ void load_pairs(const unsigned long long* src, unsign
       w[2 * h + 1] = x.y;
     }
   }
-}
-
-// Single-gap certificate: u_k the last kept logit, g the largest dropped one.
-__device__ __forceinline__ double single_gap_bound(double u_k, double g, int64_t k, int64_t n,
-                                                   int d) {
-  if (k >= n || !(g > -INFINITY)) return 0.0;
-  const double ratio = (double)k / (double)(n - k);
-  return 1.0 / (1.0 + ratio * exp((u_k - g) / sqrt((double)d)));
 }
 
 // The CTA streams V through a ring of stages; no CTA barrier is taken until
@@ -411,60 +404,10 @@ gather_kernel(const T* __restrict__ V, const float* __restrict__ u, const RowSel
     __syncthreads();
     if (s_last) {
       __threadfence();
-      if (threadIdx.x < nrows) {
-        s_wh[threadIdx.x] = sel[row0 + threadIdx.x].wh;
-        s_wt[threadIdx.x] = sel[row0 + threadIdx.x].wt;
-      }
-      // sums over the ranges, fixed order: one thread per (row, head/tail, 4 dims),
-      // 16-byte loads, eight in flight; fp64 sums staged in shared memory
-      double* fin = reinterpret_cast<double*>(red);  // [RT][2][D]
-      constexpr int NA = ERR ? 2 : 1;
-      for (int x = threadIdx.x; x < nrows * NA * (D / 4); x += kGatherThreads) {
-        const int r = x / (NA * (D / 4)), rem = x % (NA * (D / 4));
-        const int a = rem / (D / 4), d4 = rem % (D / 4);
-        const float4* src = reinterpret_cast<const float4*>(acc_out + (row0 + r) * p.nranges * 2 * D +
-                                                            a * D) + d4;
-        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-#pragma unroll 8
-        for (int c = 0; c < p.nranges; ++c) {
-          const float4 v = __ldcg(src + (int64_t)c * (2 * D / 4));
-          s0 += (double)v.x; s1 += (double)v.y; s2 += (double)v.z; s3 += (double)v.w;
-        }
-        double* f = fin + (r * 2 + a) * D + 4 * d4;
-        f[0] = s0; f[1] = s1; f[2] = s2; f[3] = s3;
-      }
-      __syncthreads();
-      // every row of the tile at once: thread x -> (row x / D, dimension x % D)
-      for (int x = threadIdx.x; x < nrows * D; x += kGatherThreads) {
-        const int r = x / D, dim = x % D;
-        const double mu_h = fin[(r * 2 + 0) * D + dim] / s_wh[r];
-        Elem<T>::store1(out + (row0 + r) * D + dim, (float)mu_h);
-        if constexpr (ERR) {
-          const double diff = s_wt[r] > 0.0 ? fin[(r * 2 + 1) * D + dim] / s_wt[r] - mu_h : 0.0;
-          fin[(r * 2 + 1) * D + dim] = diff * diff;  // each element read and rewritten by one thread
-        }
-      }
-      __syncthreads();
-      if (threadIdx.x < nrows) {  // thread r: row r's scalars
-        const int r = threadIdx.x;
-        const int64_t row = row0 + r;
-        const RowSel rs = sel[row];
-        const double wh = rs.wh, wt = rs.wt;
-        if (!(wh > 0.0)) atomicOr(status, CTA_DEV_INTERNAL);
-        if (err_out) {
-          double tot = 0.0;
-          for (int dim = 0; dim < D; ++dim) tot += fin[(r * 2 + 1) * D + dim];  // fixed order
-          err_out[row] = (float)(rs.C < rs.Z && wt > 0.0 ? rs.tv * sqrt(tot) : 0.0);
-        }
-        if (kl_out) kl_out[row] = (float)log1p(wt / wh);
-        if (gap_out) {
-          float gm = kNegInf;
-          for (int c = 0; c < p.gparts; ++c) gm = fmaxf(gm, __ldcg(gmax + row * kMaxGParts + c));
-          gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gm, rs.k, p.n,
-                                                 D);
-        }
-      }
-      __syncthreads();
+      auto sync = []() { __syncthreads(); };
+      finalize_rows<T, D, RT, ERR, kGatherThreads>(
+          threadIdx.x, sync, reinterpret_cast<double*>(red), s_wh, s_wt, acc_out, sel, gmax, out,
+          err_out, kl_out, gap_out, p, row0, nrows, status);
     }
   }
 }

@@ -49,6 +49,16 @@ cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, flo
 // dropped) keys, then (the last CTA of each (KV group, row tile), counted in
 // unit_cnt, which selection zeroes) out, err, KL and the single-gap bound.
 // gather_ctas_per_sm: the CTAs per SM its launch is planned for.
+// Phases 3 and 4 on tcgen05 for bf16 values with d = 128 (TMA-fed value
+// stages, weights as the B operand), then a row-parallel finalisation kernel
+// launched as its programmatic dependent: ranges of 128-key stages chosen by
+// set_ranges_tc(p, SM count); same outputs and workspace use as launch_gather.
+bool gather_tc_applies(const Plan& p, int dtype);
+void set_ranges_tc(Plan* p, int sms);
+cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
+                             const float* gmax, void* out, float* err_out,
+                             float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
+                             cudaStream_t st);
 int gather_ctas_per_sm(bool want_err);
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
                           uint32_t* unit_cnt, const float* gmax, void* out, float* err_out,

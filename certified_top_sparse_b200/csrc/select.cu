@@ -285,6 +285,9 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
               uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out,
               float* __restrict__ gmax, uint32_t* __restrict__ unit_cnt, Plan p,
               uint32_t* __restrict__ status) {
+  // the value pass may launch now: it streams values (independent of this
+  // kernel) and waits for its results before reading them
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();

@@ -137,6 +137,7 @@ select_short_kernel(const float* __restrict__ u, RowSel* __restrict__ sel,
                     int32_t* __restrict__ k_out, float* __restrict__ tv_out,
                     int32_t* __restrict__ idx_out, float* __restrict__ gmax,
                     uint32_t* __restrict__ unit_cnt, Plan p, uint32_t* __restrict__ status) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");  // as in the long-row kernel
   __shared__ Hist hist[kShortWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kShortWarps + warp;

@@ -87,6 +87,40 @@ def test_gqa_groups_and_query_rows(n_heads, n_kv, m):
     check(prob, 0.05, f"gqa h={n_heads} kv={n_kv} m={m}")
 
 
+# bf16 values with d = 128 take the tensor-core output pass: row tiles of 1, 2
+# and 4 rows, partial last tiles, several tiles per KV group, m > 1, ragged
+# key tails and (batch 8) several work items per CTA.
+@pytest.mark.parametrize("n_heads,n_kv,m,n", [(8, 8, 1, 2500), (8, 4, 1, 2500), (3, 1, 1, 2500),
+                                              (16, 2, 1, 2500), (6, 2, 3, 1111), (2, 2, 33, 700),
+                                              (4, 1, 1, 128), (4, 1, 1, 129), (4, 2, 1, 9999)])
+def test_gqa_groups_bf16_d128_tensor_core_values(n_heads, n_kv, m, n):
+    rng = np.random.default_rng(n_heads * 1000 + m * 10 + n)
+    d = 128
+    q = rng.standard_normal((2, n_heads, m, d)).astype(np.float32) * 1.5
+    K = rng.standard_normal((2, n_kv, n, d)).astype(np.float32)
+    V = rng.standard_normal((2, n_kv, n, d)).astype(np.float32)
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+    prob = W.Problem("gqa-bf16", bf(q), bf(K), bf(V), 0.05, 2, n_heads, n_kv, m, n, d)
+    check(prob, 0.05, f"gqa bf16 d=128 h={n_heads} kv={n_kv} m={m} n={n}")
+
+
+@pytest.mark.parametrize("want_err", [True, False])
+def test_tensor_core_values_many_items_per_cta(want_err):
+    # 64 (batch, KV head) units of 20000 keys: about four work items per CTA
+    prob = W.decode32k(batch=8, n_heads=32, n_kv_heads=8, n=20000, d=128)
+    g = gpu_run(prob, 0.01, want_err=want_err, want_kl=want_err)
+    assert g["status"] == 0
+    for b, kvh in ((0, 0), (3, 5), (7, 7)):
+        sub = sub_problem(prob, b, kvh)
+        rows = group_rows(prob, b, kvh)
+        o = run_oracle(sub, 0.01)
+        gg = {k: v for k, v in g.items()}
+        if not want_err:
+            gg["err"] = None
+            gg["kl"] = None
+        compare(sub, 0.01, gg, o, rows=rows)
+
+
 def test_bert_small_all_query():
     prob = W.bert(batch=1, n_heads=4, n=512, d=64, sharp_from=2)
     g, o, rep = check(prob, prob.eps, "bert small")
