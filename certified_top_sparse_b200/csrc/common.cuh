@@ -35,6 +35,8 @@ struct Plan {
   int range_len;        // chunks per range
   int gparts;           // partial maxima of the dropped logits per row (one per selection CTA)
   int rstages;          // tensor-core output pass: 128-key stages per range (0: not used)
+  int nmax;             // partial row maxima per row in cmax (per chunk, or per range of
+                        // the tensor-core logits pass); row stride nchunks
 };
 
 // Per-row result of the selection pass.

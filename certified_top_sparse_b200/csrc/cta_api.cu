@@ -82,6 +82,7 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   if (nchunks > kMaxChunks) return CTA_ERR_SHAPE;
   p->chunk = (int)chunk;
   p->nchunks = (int)nchunks;
+  p->nmax = (int)nchunks;
   p->scale2 = (float)(1.4426950408889634 / sqrt((double)d));  // log2(e)/sqrt(d)
   int s = 62 - ceil_log2(n);
   if (s > 52) s = 52;
@@ -167,7 +168,10 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   const bool tc = score_tc_applies(p, opts->dtype);
   // decode-shaped bf16 value sums on the tensor cores
   const bool gtc = !tc && gather_tc_applies(p, opts->dtype);
-  if (gtc) set_ranges_tc(&p, sm_count());
+  if (gtc) {
+    set_ranges_tc(&p, sm_count());
+    p.nmax = p.nranges;  // the tensor-core logits pass writes one maximum per range
+  }
   const Layout L = layout(p);
   if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
     return CTA_ERR_WORKSPACE;
@@ -185,8 +189,9 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   void** ev = opts->phase_events;
 
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
-  if ((tc ? launch_score_tc(q, K, u, p, status, st)
-          : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) != cudaSuccess)
+  if ((tc    ? launch_score_tc(q, K, u, p, status, st)
+       : gtc ? launch_score_kv_tc(q, K, u, cmax, p, status, st)
+             : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
   if ((select_short_applies(p)

@@ -418,24 +418,6 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
   }
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-
 template <int RT, bool ERR>
 cudaError_t launch_t(const CUtensorMap& map, const float* u, const RowSel* sel, float* acc,
                      const Plan& p, uint32_t* status, cudaStream_t st) {
@@ -495,6 +477,37 @@ cudaError_t launch_e(const CUtensorMap& map, const float* u, const RowSel* sel, 
 
 }  // namespace
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+
+bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc || p.d != kGD) return false;
+  // [groups][n][128] bf16: dimensions innermost, boxes of 64 dimensions x kGK keys
+  const cuuint64_t dims[3] = {(cuuint64_t)kGD, (cuuint64_t)p.n, (cuuint64_t)p.groups};
+  const cuuint64_t strides[2] = {(cuuint64_t)kGD * 2, (cuuint64_t)p.n * kGD * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)kGBox, (cuuint32_t)kGK, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool gather_tc_applies(const Plan& p, int dtype) {
   return dtype == kDtypeBF16 && p.d == kGD && p.n >= kGK && p.rt_out <= 4 && encode_tiled() != nullptr;
 }
@@ -534,18 +547,9 @@ cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, f
                              const float* gmax, void* out, float* err_out,
                              float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
                              cudaStream_t st) {
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc || p.rstages < 1) return cudaErrorInvalidValue;
-  // V as [groups][n][128] bf16: dims innermost, boxes of 64 dims x kGK keys
+  if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
-  const cuuint64_t dims[3] = {(cuuint64_t)kGD, (cuuint64_t)p.n, (cuuint64_t)p.groups};
-  const cuuint64_t strides[2] = {(cuuint64_t)kGD * 2, (cuuint64_t)p.n * kGD * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)kGBox, (cuuint32_t)kGK, 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(V), dims, strides, box, estr,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
   return p.want_err
              ? launch_e<true>(map, u, sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st)
              : launch_e<false>(map, u, sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st);

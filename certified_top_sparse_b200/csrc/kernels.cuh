@@ -1,6 +1,7 @@
 // Host-side launchers of the libcta kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -54,6 +55,14 @@ cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, flo
 // launched as its programmatic dependent: ranges of 128-key stages chosen by
 // set_ranges_tc(p, SM count); same outputs and workspace use as launch_gather.
 bool gather_tc_applies(const Plan& p, int dtype);
+// Phase 1 on tcgen05 for the same problems (bf16 q and K, d = 128), after
+// set_ranges_tc: TMA-fed K stages, the row tile's queries as the B operand;
+// writes the logits and one partial maximum per row and range (Plan::nmax).
+cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cmax, const Plan& p,
+                               uint32_t* status, cudaStream_t st);
+// Tensor map of a bf16 [groups][n][128] K or V cache: 128-byte-swizzled boxes
+// of 64 dimensions x 128 keys (the stages of the streaming tensor-core kernels).
+bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p);
 void set_ranges_tc(Plan* p, int sms);
 cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
                              const float* gmax, void* out, float* err_out,

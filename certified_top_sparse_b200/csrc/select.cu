@@ -318,9 +318,9 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   if (rank == 0 && tid == 0 && (row % p.gm) % p.rt_out == 0)
     unit_cnt[(row / p.gm) * p.tiles_out + (row % p.gm) / p.rt_out] = 0u;
 
-  // Row maximum from the per-chunk maxima of phase 1 (same in every CTA).
+  // Row maximum from the partial maxima of phase 1 (same in every CTA).
   float M = kNegInf;
-  for (int c = tid; c < p.nchunks; c += kSelThreads) M = fmaxf(M, cmax[row * p.nchunks + c]);
+  for (int c = tid; c < p.nmax; c += kSelThreads) M = fmaxf(M, cmax[row * p.nchunks + c]);
   M = block_max(M, S);
 
   for (int i = tid; i < kBins; i += kSelThreads) S.cnt[i] = 0u;
