@@ -33,7 +33,8 @@ sys.path.insert(0, ROOT)
 METRIC = "certified top-k attn query-heads/s & HBM GB/s (% of peak) at n=32K/128K"
 UNIT = "query-heads/s"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("score.cu", "select.cu", "gather.cu", "common.cuh")
+KERNEL_SOURCES = ("score.cu", "score_kv_tc.cu", "select.cu", "gather.cu", "gather_tc.cu",
+                  "finalize.cuh", "umma.cuh", "common.cuh")
 
 
 # --------------------------------------------------------------------------

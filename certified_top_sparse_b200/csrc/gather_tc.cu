@@ -376,6 +376,12 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
   const int q = tid / (2 * kGD), a = (tid / kGD) & 1, dim = tid % kGD;
+  // every load of the row is issued before the first use: the row's selection
+  // result, its dropped-logit maxima and this thread's range partials
+  const RowSel rs = sel[row];
+  float gpart = kNegInf;  // warp 2 (which forms the gap bound) loads the partial maxima
+  if (tid >= 2 * kWarp && tid - 2 * kWarp < p.gparts)
+    gpart = __ldcg(gmax + row * kMaxGParts + (tid - 2 * kWarp));
   const int per = (p.nranges + kFinQ - 1) / kFinQ;
   const int c0 = q * per, c1 = min(p.nranges, c0 + per);
   double s = 0.0;
@@ -386,7 +392,6 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
   }
   part[q][a][dim] = s;
   __syncthreads();
-  const RowSel rs = sel[row];
   if (tid < kGD) {
     double h = part[0][0][tid], t = part[0][1][tid];
 #pragma unroll
@@ -407,14 +412,15 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
     if (tid == 0) {
       if (!(rs.wh > 0.0)) atomicOr(status, CTA_DEV_INTERNAL);
       if (err_out) err_out[row] = (float)(rs.C < rs.Z && rs.wt > 0.0 ? rs.tv * sqrt(v) : 0.0);
-      if (kl_out) kl_out[row] = (float)log1p(rs.wt / rs.wh);
-      if (gap_out) {
-        float gm = kNegInf;
-        for (int c = 0; c < p.gparts; ++c) gm = fmaxf(gm, __ldcg(gmax + row * kMaxGParts + c));
-        gap_out[row] =
-            (float)single_gap_bound((double)key_value(rs.kstar), (double)gm, rs.k, p.n, kGD);
-      }
     }
+  } else if (tid == kWarp) {
+    if (kl_out) kl_out[row] = (float)log1p(rs.wt / rs.wh);
+  } else if (tid >= 2 * kWarp && tid < 3 * kWarp && gap_out) {
+    // the row's largest dropped logit over the selection CTAs' partial maxima
+    float gm = __shfl_sync(0xffffffffu, gpart, 0);
+    for (int c = 1; c < kMaxGParts; ++c) gm = fmaxf(gm, __shfl_sync(0xffffffffu, gpart, c));
+    if (tid == 2 * kWarp)
+      gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gm, rs.k, p.n, kGD);
   }
 }
 

@@ -10,6 +10,7 @@ import csv
 import io
 import json
 import os
+import re
 import subprocess
 import sys
 
@@ -29,8 +30,9 @@ def main(rep, command):
     out = {}
     for r in data:
         name = r[col["Kernel Name"]]
-        key = next((k for k in ("score", "select", "gather", "finalize") if f"{k}_kernel" in name),
-                   None)
+        # score[_kv_tc]_kernel, select_kernel, gather[_tc]_kernel, finalize_tc_kernel
+        key = next((k for k in ("score", "select", "gather", "finalize")
+                    if re.search(rf"\b{k}(_kv)?(_tc)?_kernel\b", name)), None)
         if key is None:
             continue
         rd = float(r[col["dram__bytes_read.sum"]]) * scale[units[col["dram__bytes_read.sum"]]]
