@@ -605,19 +605,25 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
         msum += ms[j];
         csum += cs[j];
       }
-      unsigned long long tmp;
-      unsigned long long cum = c_above + block_scan_excl(msum, &tmp, S);
-      unsigned long long cnt_before = block_scan_excl(csum, &tmp, S);
+      unsigned long long sc[3] = {msum, csum, 0ull}, stot[3];
+      block_scan_excl3(sc, stot, S);
+      unsigned long long cum = c_above + sc[0];
+      unsigned long long cnt_before = sc[1];
+      // The certificate holds from one sub-bin on (the cumulative mass only
+      // grows): only the thread whose sub-bins contain the change searches.
+      if (!certified(Z, cum, p.eps) && certified(Z, cum + msum, p.eps)) {
 #pragma unroll
-      for (int j = 0; j < SPT; ++j) {
-        const int sb = tid * SPT + j;
-        if (sb < nsub && certified(Z, cum + ms[j], p.eps) && !certified(Z, cum, p.eps)) {
-          S.pos = sb;
-          S.c_above = cum;            // mass ranked above the sub-bin
-          S.n_above = cnt_before;     // window keys ranked above it
+        for (int j = 0; j < SPT; ++j) {
+          const int sb = tid * SPT + j;
+          if (sb < nsub && certified(Z, cum + ms[j], p.eps)) {
+            S.pos = sb;
+            S.c_above = cum;            // mass ranked above the sub-bin
+            S.n_above = cnt_before;     // window keys ranked above it
+            break;
+          }
+          cum += ms[j];
+          cnt_before += cs[j];
         }
-        cum += ms[j];
-        cnt_before += cs[j];
       }
       __syncthreads();
       const int sstar = S.pos;
@@ -685,14 +691,18 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
     }
     unsigned long long tmp;
     unsigned long long cum = base_mass + block_scan_excl(wsum, &tmp, S);
+    // as for the sub-bins: the certificate changes once along the sorted keys
+    if (!certified(Z, cum, p.eps) && certified(Z, cum + wsum, p.eps)) {
 #pragma unroll
-    for (int j = 0; j < E; ++j) {
-      const int i = tid * E + j;
-      if (i < m && certified(Z, cum + wloc[j], p.eps) && !certified(Z, cum, p.eps)) {
-        S.pos = i;
-        S.c_above = cum + wloc[j];  // kept mass C_k
+      for (int j = 0; j < E; ++j) {
+        const int i = tid * E + j;
+        if (i < m && certified(Z, cum + wloc[j], p.eps)) {
+          S.pos = i;
+          S.c_above = cum + wloc[j];  // kept mass C_k
+          break;
+        }
+        cum += wloc[j];
       }
-      cum += wloc[j];
     }
     __syncthreads();
     int pos = S.pos;
@@ -714,6 +724,21 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
         atomicAdd(&cc[idx / chunk], 1u);
       }
     }
+    // the CTAs' fp64 sums of the weights above / below the window: loaded by
+    // warp 0 in parallel, added in rank order
+    double fa_row = 0.0, fb_row = 0.0;
+    if (warp == 0) {
+      double x0 = 0.0, x1 = 0.0;
+      if (lane < CS) {
+        const SelShared* R = cluster.map_shared_rank(&S, lane);
+        x0 = R->fpart[0];
+        x1 = R->fpart[1];
+      }
+      for (int q = 0; q < CS; ++q) {
+        fa_row += __shfl_sync(0xffffffffu, x0, q);
+        fb_row += __shfl_sync(0xffffffffu, x1, q);
+      }
+    }
     if (tid == 0) {
       long long k = (long long)base_cnt + pos + 1;
       if (k > n) k = n;
@@ -731,12 +756,6 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
       r.tv = Z ? (double)(Z - C) / (double)Z : 0.0;
       // kept = above the window + the window's kept candidates; dropped likewise
       // (an oversized window recomputes both in the recount pass below)
-      double fa_row = 0.0, fb_row = 0.0;
-      for (int q = 0; q < CS; ++q) {
-        const SelShared* R = cluster.map_shared_rank(&S, q);
-        fa_row += R->fpart[0];
-        fb_row += R->fpart[1];
-      }
       r.wh = fa_row + S.fsum[0];
       r.wt = fb_row + S.fsum[1];
       sel[row] = r;
