@@ -53,7 +53,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kSubPerBin = 64;          // sub-bins per bin: 4096 per halving of the weight
 constexpr int kSub = 2048;              // sub-bins available (a window of up to 32 bins)
 constexpr int kLocalChunks = 1024;      // per-CTA chunk counters kept in shared memory
-constexpr int kIdxBatch = 16;           // 32-key words in flight per warp in the index pass
+constexpr int kIdxBatch = 20;           // 32-key words in flight per warp in the index pass
 constexpr int kBinsPerThread = kBins / kSelThreads;
 constexpr double kBoundSlack = 4e-6;    // covers exp2f's error (2 ulp) with margin
 constexpr double kDecideSlack = 1e-9;   // covers fp64 rounding in the exact test
