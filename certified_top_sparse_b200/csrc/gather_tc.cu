@@ -370,6 +370,9 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
                    const float* __restrict__ gmax, __nv_bfloat16* __restrict__ out,
                    float* __restrict__ err_out, float* __restrict__ kl_out,
                    float* __restrict__ gap_out, Plan p, uint32_t* __restrict__ status) {
+  // The next call's logits pass may be scheduled now (it streams K at once
+  // and waits for this grid before it writes the logits).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ double part[kFinQ][2][kGD];
   __shared__ double sq[kGD];

@@ -210,6 +210,11 @@ score_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16
   } else {
     // ---------------- epilogue ----------------
     const int tid = threadIdx.x - kSEpiWarp0 * kWarp;  // 0..127
+    // Launched as a programmatic dependent of the kernel before it in the
+    // stream (the previous call's finalisation): K and q are inputs and stream
+    // at once; the logit buffer and maxima are written only after that grid
+    // (and with it the value pass that reads the logits) has finished.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int quarter = warp & 3;                      // TMEM lanes (keys) this warp may read
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
     int t = 0;
@@ -291,9 +296,18 @@ cudaError_t launch_t(const CUtensorMap& map, const void* q, float* u, float* cma
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long nitems = (long long)p.tiles_score * p.nranges * p.groups;
   const unsigned grid = (unsigned)std::min<long long>(nitems, sms);
-  kern<<<grid, kSThreads, kSSmem, st>>>(map, static_cast<const __nv_bfloat16*>(q), u, cmax, p,
-                                        status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kSThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see the epilogue
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, map, static_cast<const __nv_bfloat16*>(q), u, cmax, p,
+                            status);
 }
 
 }  // namespace

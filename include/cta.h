@@ -25,6 +25,14 @@
  *     argument and launch errors only.  Conditions found on the device (a
  *     non-finite logit, a broken internal invariant) are OR-ed as bits into
  *     *cta_opts.status_dev when that pointer is given.  No device code traps.
+ *   - For bf16 inputs with d = 128 the kernels of a call are launched with
+ *     programmatic stream serialization: the first one may start reading q
+ *     and K while the kernel before it on the stream finishes, if that kernel
+ *     lets its dependents launch early (griddepcontrol.launch_dependents);
+ *     it writes nothing before that kernel has completed.  A caller's kernel
+ *     that triggers its dependents early must not write q or K after the
+ *     trigger.  Kernels that never trigger (the usual case) and copies give
+ *     ordinary stream order.
  *   - Supported: d in {64, 128}; 1 <= n <= 2^28; 0 < eps < 1;
  *     n_heads % n_kv_heads == 0; batch, m >= 1.  There is no mask: every row
  *     sees all n keys.  The logit scale is 1/sqrt(d).
