@@ -357,12 +357,12 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
 }
 
 // Phase 4: one CTA per row, launched as a programmatic dependent of the value
-// pass (it waits for that grid's results).  Thread (q, a, dim) sums range
-// quarter q of the head (a = 0) or tail (a = 1) partials of one dimension with
-// every load in flight; the quarters are then added in a fixed order, so the
-// result does not depend on timing.
-constexpr int kFinQ = 4;
-constexpr int kFinThreads = kFinQ * 2 * kGD;
+// pass (it waits for that grid's results).  Thread (a, dim) sums the head
+// (a = 0) or tail (a = 1) partials of one dimension over the ranges in a fixed
+// order, sixteen loads in flight.  256 threads: the CTA fits beside a value-
+// pass or logits CTA on an SM, so it neither waits for a free SM nor keeps the
+// next call's logits pass off one.
+constexpr int kFinThreads = 2 * kGD;
 
 template <bool ERR>
 __global__ void __launch_bounds__(kFinThreads)
@@ -374,38 +374,30 @@ finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__
   // and waits for this grid before it writes the logits).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ double part[kFinQ][2][kGD];
+  __shared__ double tail[kGD];
   __shared__ double sq[kGD];
   const int64_t row = blockIdx.x;
   const int tid = threadIdx.x;
-  const int q = tid / (2 * kGD), a = (tid / kGD) & 1, dim = tid % kGD;
+  const int a = tid / kGD, dim = tid % kGD;
   // every load of the row is issued before the first use: the row's selection
   // result, its dropped-logit maxima and this thread's range partials
   const RowSel rs = sel[row];
   float gpart = kNegInf;  // warp 2 (which forms the gap bound) loads the partial maxima
   if (tid >= 2 * kWarp && tid - 2 * kWarp < p.gparts)
     gpart = __ldcg(gmax + row * kMaxGParts + (tid - 2 * kWarp));
-  const int per = (p.nranges + kFinQ - 1) / kFinQ;
-  const int c0 = q * per, c1 = min(p.nranges, c0 + per);
   double s = 0.0;
   if (ERR || a == 0) {
     const float* src = acc_out + (row * p.nranges * 2 + a) * kGD + dim;
 #pragma unroll 16
-    for (int c = c0; c < c1; ++c) s += (double)__ldcg(src + (int64_t)c * 2 * kGD);
+    for (int c = 0; c < p.nranges; ++c) s += (double)__ldcg(src + (int64_t)c * 2 * kGD);
   }
-  part[q][a][dim] = s;
+  if (a == 1) tail[dim] = s;
   __syncthreads();
-  if (tid < kGD) {
-    double h = part[0][0][tid], t = part[0][1][tid];
-#pragma unroll
-    for (int qq = 1; qq < kFinQ; ++qq) {
-      h += part[qq][0][tid];
-      t += part[qq][1][tid];
-    }
-    const double mu_h = h / rs.wh;
-    out[row * kGD + tid] = __float2bfloat16_rn((float)mu_h);
-    const double diff = (ERR && rs.wt > 0.0) ? t / rs.wt - mu_h : 0.0;
-    sq[tid] = diff * diff;
+  if (a == 0) {
+    const double mu_h = s / rs.wh;
+    out[row * kGD + dim] = __float2bfloat16_rn((float)mu_h);
+    const double diff = (ERR && rs.wt > 0.0) ? tail[dim] / rs.wt - mu_h : 0.0;
+    sq[dim] = diff * diff;
   }
   __syncthreads();
   if (tid < kWarp) {  // fixed-order tree over the dimensions

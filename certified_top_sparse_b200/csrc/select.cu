@@ -285,8 +285,11 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
               uint32_t* __restrict__ chunk_off, int32_t* __restrict__ idx_out,
               float* __restrict__ gmax, uint32_t* __restrict__ unit_cnt, Plan p,
               uint32_t* __restrict__ status) {
-  // the value pass may launch now: it streams values (independent of this
-  // kernel) and waits for its results before reading them
+  // Launched as a programmatic dependent of the logits pass (which does not
+  // trigger early, so this only saves the launch latency): wait for it, then
+  // let the value pass launch (it streams values, which do not depend on this
+  // kernel, and waits for its results before reading them).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(smem_raw);
@@ -872,13 +875,15 @@ cudaError_t launch_select(const float* u, const float* cmax, RowSel* sel, int32_
   cfg.blockDim = dim3(kSelThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)p.sel_cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see the kernel's first lines
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, select_kernel, u, cmax, sel, k_out, tv_out, chunk_off, idx_out, gmax,
                          unit_cnt, p, status);
   if (e != cudaSuccess) return e;
