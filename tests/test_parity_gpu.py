@@ -121,6 +121,34 @@ def test_tensor_core_values_many_items_per_cta(want_err):
         compare(sub, 0.01, gg, o, rows=rows)
 
 
+@pytest.mark.parametrize("want_err", [True, False])
+def test_back_to_back_calls_share_one_workspace(want_err):
+    # Calls issued back to back on one stream with one workspace and no host
+    # synchronisation between them: the next call's logits pass overlaps this
+    # call's finalisation and the value pass starts during selection.  Every
+    # call must still match the oracle.
+    prob = W.decode128k(batch=1, n=40000, steps=4)
+    dev = torch.device("cuda")
+    K, V = prob.K.to(dev), prob.V.to(dev)
+    qs = prob.meta["q_steps"].to(dev)
+    ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                            batch=prob.batch), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    results = []
+    for t in range(4):
+        results.append(cta.cta_certified_topk_attn(qs[t], K, V, 0.01, workspace=ws,
+                                                   status_dev=status, want_err=want_err,
+                                                   want_kl=want_err, want_gap=True))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for t in range(4):
+        g = to_host(results[t])
+        for kvh in (0, 5):
+            sub = sub_problem(prob, 0, kvh, q=prob.meta["q_steps"][t])
+            o = run_oracle(sub, 0.01)
+            compare(sub, 0.01, g, o, rows=group_rows(prob, 0, kvh))
+
+
 def test_bert_small_all_query():
     prob = W.bert(batch=1, n_heads=4, n=512, d=64, sharp_from=2)
     g, o, rep = check(prob, prob.eps, "bert small")
