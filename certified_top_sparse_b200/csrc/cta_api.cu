@@ -206,11 +206,15 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
                      st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+  } else if (gtc) {  // tensor-core value sums, then the row-parallel finalisation
+    if (launch_gather_tc(V, u, sel, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (launch_finalize_tc(acc, sel, gmax, out, opts->err_out, opts->kl_out, opts->gap_out, p,
+                           status, st) != cudaSuccess)
+      return CTA_ERR_CUDA;
   } else {  // value sums, then the last CTA of each row tile finalises it
-    if ((gtc ? launch_gather_tc(V, u, sel, acc, gmax, out, opts->err_out, opts->kl_out,
-                                opts->gap_out, p, status, st)
-             : launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
-                             opts->kl_out, opts->gap_out, p, status, st)) != cudaSuccess)
+    if (launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
+                      opts->kl_out, opts->gap_out, p, status, st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
   }

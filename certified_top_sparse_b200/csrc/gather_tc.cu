@@ -463,17 +463,13 @@ cudaError_t launch_finalize(const float* acc, const RowSel* sel, const float* gm
 
 template <bool ERR>
 cudaError_t launch_e(const CUtensorMap& map, const float* u, const RowSel* sel, float* acc,
-                     const float* gmax, void* out, float* err_out, float* kl_out, float* gap_out,
                      const Plan& p, uint32_t* status, cudaStream_t st) {
-  cudaError_t e;
   switch (p.rt_out) {
-    case 1: e = launch_t<1, ERR>(map, u, sel, acc, p, status, st); break;
-    case 2: e = launch_t<2, ERR>(map, u, sel, acc, p, status, st); break;
-    case 4: e = launch_t<4, ERR>(map, u, sel, acc, p, status, st); break;
+    case 1: return launch_t<1, ERR>(map, u, sel, acc, p, status, st);
+    case 2: return launch_t<2, ERR>(map, u, sel, acc, p, status, st);
+    case 4: return launch_t<4, ERR>(map, u, sel, acc, p, status, st);
     default: return cudaErrorInvalidValue;
   }
-  if (e != cudaSuccess) return e;
-  return launch_finalize<ERR>(acc, sel, gmax, out, err_out, kl_out, gap_out, p, status, st);
 }
 
 }  // namespace
@@ -545,15 +541,20 @@ void set_ranges_tc(Plan* p, int sms) {
 }
 
 cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
-                             const float* gmax, void* out, float* err_out,
-                             float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
-                             cudaStream_t st) {
+                             const Plan& p, uint32_t* status, cudaStream_t st) {
   if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
   if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
+  return p.want_err ? launch_e<true>(map, u, sel, acc, p, status, st)
+                    : launch_e<false>(map, u, sel, acc, p, status, st);
+}
+
+cudaError_t launch_finalize_tc(const float* acc, const RowSel* sel, const float* gmax, void* out,
+                               float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                               uint32_t* status, cudaStream_t st) {
   return p.want_err
-             ? launch_e<true>(map, u, sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st)
-             : launch_e<false>(map, u, sel, acc, gmax, out, err_out, kl_out, gap_out, p, status, st);
+             ? launch_finalize<true>(acc, sel, gmax, out, err_out, kl_out, gap_out, p, status, st)
+             : launch_finalize<false>(acc, sel, gmax, out, err_out, kl_out, gap_out, p, status, st);
 }
 
 }  // namespace cta

@@ -50,10 +50,10 @@ cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, flo
 // dropped) keys, then (the last CTA of each (KV group, row tile), counted in
 // unit_cnt, which selection zeroes) out, err, KL and the single-gap bound.
 // gather_ctas_per_sm: the CTAs per SM its launch is planned for.
-// Phases 3 and 4 on tcgen05 for bf16 values with d = 128 (TMA-fed value
-// stages, weights as the B operand), then a row-parallel finalisation kernel
-// launched as its programmatic dependent: ranges of 128-key stages chosen by
-// set_ranges_tc(p, SM count); same outputs and workspace use as launch_gather.
+// Phase 3 on tcgen05 for bf16 values with d = 128 (TMA-fed value stages,
+// weights as the B operand), ranges of 128-key stages chosen by
+// set_ranges_tc(p, SM count); the range partials go to acc as in
+// launch_gather, and launch_finalize_tc forms the outputs.
 bool gather_tc_applies(const Plan& p, int dtype);
 // Phase 1 on tcgen05 for the same problems (bf16 q and K, d = 128), after
 // set_ranges_tc: TMA-fed K stages, the row tile's queries as the B operand;
@@ -65,9 +65,11 @@ cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cm
 bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p);
 void set_ranges_tc(Plan* p, int sms);
 cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
-                             const float* gmax, void* out, float* err_out,
-                             float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
-                             cudaStream_t st);
+                             const Plan& p, uint32_t* status, cudaStream_t st);
+// Phase 4 after launch_gather_tc: one CTA per row, a programmatic dependent of it.
+cudaError_t launch_finalize_tc(const float* acc, const RowSel* sel, const float* gmax, void* out,
+                               float* err_out, float* kl_out, float* gap_out, const Plan& p,
+                               uint32_t* status, cudaStream_t st);
 int gather_ctas_per_sm(bool want_err);
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
                           uint32_t* unit_cnt, const float* gmax, void* out, float* err_out,
