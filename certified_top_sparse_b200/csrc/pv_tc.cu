@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "umma.cuh"
 
 namespace cta {
 
@@ -30,65 +31,7 @@ namespace {
 constexpr int kPvRows = 128;      // M: query rows per CTA (TMEM lanes)
 constexpr int kPvKeys = 64;       // keys per chunk: one 128-byte swizzle atom of bf16
 constexpr int kPvThreads = 256;   // two threads per row
-constexpr int kRowB = 128;
-constexpr int kATile = kPvRows * kRowB;  // one A matrix of a chunk: 128 rows x 64 bf16 = 16 KB
-
-__device__ __forceinline__ uint32_t swz(int r, int c, int rows) {
-  const int atom = c >> 3, cc = c & 7;
-  return (uint32_t)(atom * rows * kRowB + (r >> 3) * 1024 + (r & 7) * kRowB + ((cc ^ (r & 7)) << 4));
-}
-// K-major, 128-byte swizzle: SBO 1024 B, LBO 16 B (unused), version 1.
-__device__ __forceinline__ unsigned long long desc_k(uint32_t saddr) {
-  return (unsigned long long)((saddr >> 4) & 0x3FFFu) | (1ull << 16) |
-         ((unsigned long long)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-// MN-major, 128-byte swizzle: 8-key groups 1024 B apart (SBO), 64-dim blocks
-// lbo bytes apart (LBO), version 1.
-__device__ __forceinline__ unsigned long long desc_mn(uint32_t saddr, uint32_t lbo) {
-  return (unsigned long long)((saddr >> 4) & 0x3FFFu) |
-         ((unsigned long long)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((unsigned long long)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-// kind::f16, A, B bf16, D fp32, A K-major, B MN-major, M x N.
-constexpr uint32_t idesc_pv(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, unsigned long long a, unsigned long long b,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
-      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(unsigned long long* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* v) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
+constexpr int kATile = kPvRows * kSwRowBytes;  // one A matrix of a chunk: 128 rows x 64 bf16 = 16 KB
 
 // bf16 hi/lo parts of two weights, packed (lower key in the low half).
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
@@ -131,11 +74,7 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
   const int r = threadIdx.x % kPvRows;   // this thread's row (TMEM lane)
   const int half = threadIdx.x / kPvRows;  // which 32 keys of a chunk it converts
 
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(&tmem_slot)), "r"(S::kCols) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 0) tmem_alloc(&tmem_slot, S::kCols);
   if (threadIdx.x == 0) {
     mbar_init(&done[0], 1);
     mbar_init(&done[1], 1);
@@ -148,7 +87,7 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
-  constexpr uint32_t idesc = idesc_pv(kPvRows, D);
+  constexpr uint32_t idesc = idesc_bf16(kPvRows, D, /*a_mn=*/false, /*b_mn=*/true);
   const int nch = (int)(p.n / kPvKeys);
   bool ok = true;
 
@@ -206,7 +145,7 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
           split2(kh[0], kh[1], hh[e], hl[e]);
           if constexpr (ERR) split2(kd[0], kd[1], th[e], tl[e]);
         }
-        const uint32_t off = swz(r, half * 4 + c, kPvRows);
+        const uint32_t off = sw128_offset(r, half * 4 + c, kPvRows);
         *reinterpret_cast<uint4*>(ab + 0 * kATile + off) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
         *reinterpret_cast<uint4*>(ab + 1 * kATile + off) = make_uint4(hl[0], hl[1], hl[2], hl[3]);
         if constexpr (ERR) {
@@ -219,23 +158,23 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int q = threadIdx.x + i * kPvThreads, key = q / P, c = q % P;
-      *reinterpret_cast<uint4*>(vb + swz(key, c, kPvKeys)) = vv[i];
+      *reinterpret_cast<uint4*>(vb + sw128_offset(key, c, kPvKeys)) = vv[i];
     }
     fence_proxy_async();
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
       const uint32_t a0 = smem_u32(ab), v0 = smem_u32(vb);
-      constexpr uint32_t lbo = kPvKeys * kRowB;  // 64-dim blocks of V, 8 KB apart
+      constexpr uint32_t lbo = kPvKeys * kSwRowBytes;  // 64-dim blocks of V, 8 KB apart
 #pragma unroll
       for (int s = 0; s < kPvKeys / 16; ++s) {
-        const unsigned long long bd = desc_mn(v0 + (uint32_t)(s * 2048), lbo);
+        const unsigned long long bd = desc_mnmajor(v0 + (uint32_t)(s * 2048), lbo);
         const uint32_t acc = (j > 0 || s > 0) ? 1u : 0u;
-        tc_mma(tmem, desc_k(a0 + 0 * kATile + s * 32), bd, idesc, acc);
-        tc_mma(tmem, desc_k(a0 + 1 * kATile + s * 32), bd, idesc, 1u);
+        tc_mma(tmem, desc_kmajor(a0 + 0 * kATile + s * 32), bd, idesc, acc);
+        tc_mma(tmem, desc_kmajor(a0 + 1 * kATile + s * 32), bd, idesc, 1u);
         if constexpr (ERR) {
-          tc_mma(tmem + D, desc_k(a0 + 2 * kATile + s * 32), bd, idesc, acc);
-          tc_mma(tmem + D, desc_k(a0 + 3 * kATile + s * 32), bd, idesc, 1u);
+          tc_mma(tmem + D, desc_kmajor(a0 + 2 * kATile + s * 32), bd, idesc, acc);
+          tc_mma(tmem + D, desc_kmajor(a0 + 3 * kATile + s * 32), bd, idesc, 1u);
         }
       }
       tc_commit(&done[b]);
@@ -301,9 +240,7 @@ pv_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::kCols)
-                 : "memory");
+  if (warp == 0) tmem_dealloc(tmem, S::kCols);
 }
 
 template <int D, bool ERR>

@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "umma.cuh"
 
 namespace cta {
 
@@ -28,67 +29,6 @@ namespace {
 constexpr int kTcRows = 128;     // M: query rows per CTA (one per thread and TMEM lane)
 constexpr int kTcN = 256;        // N: keys per MMA chunk (TMEM columns)
 constexpr int kTcThreads = 256;  // two warpgroups: same TMEM lanes (rows), half the columns each
-constexpr int kAtomRows = 8;     // rows per 128-byte swizzle atom
-constexpr int kRowBytes = 128;   // one atom row: 64 bf16 of K (the contraction dim)
-
-// Byte offset of 16-byte piece c (c < d/8) of row r in a K-major, 128-byte
-// swizzled tile of `rows` rows: d/64 column atoms of rows x 128 B, each made
-// of 8-row groups of 1024 B in which piece c of row r sits at c ^ (r % 8).
-__device__ __forceinline__ uint32_t sw128_offset(int r, int c, int rows) {
-  const int atom = c >> 3, cc = c & 7;
-  return (uint32_t)(atom * rows * kRowBytes + (r >> 3) * (kAtomRows * kRowBytes) +
-                    (r & 7) * kRowBytes + ((cc ^ (r & 7)) << 4));
-}
-
-// Shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle, 8-row
-// groups 1024 B apart (stride byte offset), leading byte offset 16 (unused for
-// swizzled K-major), descriptor version 1.
-__device__ __forceinline__ unsigned long long sw128_desc(uint32_t saddr) {
-  return (unsigned long long)((saddr >> 4) & 0x3FFFu) | (1ull << 16) |
-         ((unsigned long long)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor: kind::f16, A and B bf16 (K-major), D fp32, M x N.
-constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, unsigned long long a, unsigned long long b,
-                                       uint32_t idesc, bool accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
-      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(unsigned long long* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               ::"r"(smem_u32(bar)) : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t* v) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
-      "%28, %29, %30, %31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // Stages rows [0, rows) of a row-major [*, D] bf16 matrix into the swizzled tile.
 template <int D>
@@ -121,11 +61,7 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   const int group = blockIdx.x / tiles, tile = blockIdx.x % tiles;
   const int64_t row0 = (int64_t)group * p.gm + (int64_t)tile * kTcRows;
 
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(&tmem_slot)), "r"(kTcN) : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 0) tmem_alloc(&tmem_slot, kTcN);
   if (threadIdx.x == 0) {
     mbar_init(&mma_done, 1);
     mbar_fence_init();
@@ -138,7 +74,7 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
   const __nv_bfloat16* Kg = K + (int64_t)group * p.n * D;
   float* urow = u + (row0 + rr) * p.ustride;
-  constexpr uint32_t idesc = idesc_bf16_f32(kTcRows, kTcN);
+  constexpr uint32_t idesc = idesc_bf16(kTcRows, kTcN, false, false);
   bool ok = true;
 
   const int nchunks = (int)(p.n / kTcN);
@@ -152,9 +88,9 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
       for (int s = 0; s < D / 16; ++s) {
         // k-step s: atom s / 4, 32-byte slice s % 4 of each 128-byte row
         const uint32_t off = (uint32_t)((s & 3) * 32);
-        const uint32_t qa = smem_u32(qs) + (uint32_t)((s >> 2) * kTcRows * kRowBytes) + off;
-        const uint32_t ka = smem_u32(ks) + (uint32_t)((s >> 2) * kTcN * kRowBytes) + off;
-        tc_mma(tmem, sw128_desc(qa), sw128_desc(ka), idesc, s > 0);
+        const uint32_t qa = smem_u32(qs) + (uint32_t)((s >> 2) * kTcRows * kSwRowBytes) + off;
+        const uint32_t ka = smem_u32(ks) + (uint32_t)((s >> 2) * kTcN * kSwRowBytes) + off;
+        tc_mma(tmem, desc_kmajor(qa), desc_kmajor(ka), idesc, s > 0);
       }
       tc_commit(&mma_done);
     }
@@ -180,9 +116,7 @@ score_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     if (__syncthreads_or(ok ? 0 : 1)) break;
   }
   tc_fence_after();
-  if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTcN)
-                 : "memory");
+  if (warp == 0) tmem_dealloc(tmem, kTcN);
 }
 
 template <int D>
