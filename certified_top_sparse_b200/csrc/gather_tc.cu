@@ -512,23 +512,50 @@ bool gather_tc_applies(const Plan& p, int dtype) {
 void set_ranges_tc(Plan* p, int sms) {
   const int64_t units = (int64_t)p->groups * p->tiles_out;
   const int64_t spu = (p->n + kGK - 1) / kGK;
-  const int64_t cap = std::min<int64_t>(spu, p->nchunks);  // range partials fit the workspace
-  constexpr int64_t kItemCost = 2;  // stages' worth of fill and hand-over per item
-  int64_t best = -1, best_rs = spu, best_nr = 1;
-  for (int k = 1; k <= 4; ++k) {
-    int64_t nr = ((int64_t)k * sms + units - 1) / units;
-    nr = std::max<int64_t>(1, std::min(nr, cap));
+  // range partials fit the workspace (one slot per chunk); at most 1024 ranges are tried
+  const int64_t cap = std::min<int64_t>(std::min<int64_t>(spu, p->nchunks), 1024);
+  constexpr int64_t kItemCost = 1;  // a stage's worth of hand-over per item
+  // Every range count is scored by the busiest CTA's items times their length
+  // (items go round-robin over the grid); the eight best are then simulated
+  // exactly (the last range of a unit is shorter).
+  constexpr int kTry = 8;
+  int64_t cand[kTry], cscore[kTry];
+  int ncand = 0;
+  for (int64_t nr = 1; nr <= cap; ++nr) {
     const int64_t rs = (spu + nr - 1) / nr;
     const int64_t nranges = (spu + rs - 1) / rs;
+    if (nranges != nr) continue;  // the same cut as a smaller count
+    const int64_t items = units * nranges;
+    const int64_t G = std::min<int64_t>(items, sms);
+    const int64_t score = (items + G - 1) / G * (rs + kItemCost);
+    int at;
+    if (ncand < kTry) {
+      at = ncand++;
+    } else {
+      if (score >= cscore[kTry - 1]) continue;
+      at = kTry - 1;
+    }
+    cand[at] = nr;
+    cscore[at] = score;
+    while (at > 0 && cscore[at] < cscore[at - 1]) {  // keep the list sorted by score
+      std::swap(cand[at], cand[at - 1]);
+      std::swap(cscore[at], cscore[at - 1]);
+      --at;
+    }
+  }
+  int64_t best = -1, best_rs = spu, best_nr = 1;
+  for (int c = 0; c < ncand; ++c) {
+    const int64_t nranges = cand[c];
+    const int64_t rs = (spu + nranges - 1) / nranges;
     const int64_t last = spu - (nranges - 1) * rs;
     const int64_t items = units * nranges;
     const int64_t G = std::min<int64_t>(items, sms);
     int64_t worst = 0;  // stages of the busiest CTA (items b, b + G, ... of the grid)
     for (int64_t b = 0; b < G; ++b) {
-      int64_t c = 0;
+      int64_t w = 0;
       for (int64_t i = b; i < items; i += G)
-        c += (((i / p->tiles_out) % nranges) == nranges - 1 ? last : rs) + kItemCost;
-      worst = std::max(worst, c);
+        w += (((i / p->tiles_out) % nranges) == nranges - 1 ? last : rs) + kItemCost;
+      worst = std::max(worst, w);
     }
     if (best < 0 || worst < best) {
       best = worst;
