@@ -116,18 +116,25 @@ Layout layout(const Plan& p) {
 
 bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
-
 int record(void** ev, int i, cudaStream_t st) {
   if (!ev) return CTA_OK;
   return cudaEventRecord((cudaEvent_t)ev[i], st) == cudaSuccess ? CTA_OK : CTA_ERR_CUDA;
 }
 
 }  // namespace
+int g_sm_count[64];  // per device, filled on first use (every thread writes the same value)
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_sm_count[dev] == 0) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+    g_sm_count[dev] = c;
+  }
+  return g_sm_count[dev];
+}
+
 }  // namespace cta
 
 using namespace cta;

@@ -432,8 +432,7 @@ cudaError_t launch_gather_t(const void* V, const float* u, const RowSel* sel, co
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGatherThreads, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const long long nitems = (long long)p.tiles_out * p.nranges * p.groups;
   const long long grid = std::min<long long>(nitems, (long long)std::max(per_sm, 1) * sms);
   kern<<<(unsigned)grid, kGatherThreads, smem, st>>>(

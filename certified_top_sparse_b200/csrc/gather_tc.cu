@@ -425,8 +425,7 @@ cudaError_t launch_t(const CUtensorMap& map, const float* u, const RowSel* sel, 
   auto kern = gather_tc_kernel<RT, ERR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const long long nitems = (long long)p.tiles_out * p.nranges * p.groups;
   const unsigned grid = (unsigned)std::min<long long>(nitems, sms);
   // programmatic dependent of selection: the value stream starts early

@@ -13,6 +13,9 @@ namespace cta {
 constexpr int kDtypeF32 = CTA_F32;
 constexpr int kDtypeBF16 = CTA_BF16;
 
+// SMs of the current device (cached per device; 148 if the query fails).
+int sm_count();
+
 // Phase 1: logits u [rows, n] and per-(row, chunk) maxima cmax [rows, nchunks].
 cudaError_t launch_score(int dtype, const void* q, const void* K, float* u, float* cmax,
                          const Plan& p, uint32_t* status, cudaStream_t st);

@@ -283,19 +283,6 @@ score_kernel(const T* __restrict__ q, const T* __restrict__ K, float* __restrict
   }
 }
 
-int g_sm_count[64];
-
-int sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (g_sm_count[dev] == 0) {
-    int c = 0;
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
-    g_sm_count[dev] = c;
-  }
-  return g_sm_count[dev];
-}
-
 template <typename T, int D, int RT>
 cudaError_t launch_score_t(const void* q, const void* K, float* u, float* cmax, const Plan& p,
                            uint32_t* status, cudaStream_t st) {

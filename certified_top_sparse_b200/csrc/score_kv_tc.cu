@@ -292,8 +292,7 @@ cudaError_t launch_t(const CUtensorMap& map, const void* q, float* u, float* cma
   auto kern = score_kv_tc_kernel<RT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSSmem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const long long nitems = (long long)p.tiles_score * p.nranges * p.groups;
   const unsigned grid = (unsigned)std::min<long long>(nitems, sms);
   cudaLaunchConfig_t cfg = {};
