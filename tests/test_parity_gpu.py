@@ -104,6 +104,18 @@ def test_gqa_groups_bf16_d128_tensor_core_values(n_heads, n_kv, m, n):
     check(prob, 0.05, f"gqa bf16 d=128 h={n_heads} kv={n_kv} m={m} n={n}")
 
 
+@pytest.mark.parametrize("n", [1, 17, 100, 127])
+def test_bf16_d128_shorter_than_one_stage(n):
+    # fewer keys than one 128-key tensor-core stage: the CUDA-core kernels take over
+    rng = np.random.default_rng(7000 + n)
+    d = 128
+    bf = lambda a: torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16)
+    q = bf(rng.standard_normal((1, 8, 1, d)) * 1.5)
+    K, V = bf(rng.standard_normal((1, 2, n, d))), bf(rng.standard_normal((1, 2, n, d)))
+    prob = W.Problem("short-bf16", q, K, V, 0.05, 1, 8, 2, 1, n, d)
+    check(prob, 0.05, f"bf16 d=128 n={n}")
+
+
 @pytest.mark.parametrize("want_err", [True, False])
 def test_tensor_core_values_many_items_per_cta(want_err):
     # 64 (batch, KV head) units of 20000 keys: about four work items per CTA
