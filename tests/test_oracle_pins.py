@@ -250,8 +250,30 @@ def test_two_keys_closed_form():
                 assert r["k"][0] == 1 and r["idx"][0].tolist() == ([1] if D > 0 else [0])
                 assert r["tv"][0] == pytest.approx(p_small, rel=1e-13)
                 assert r["err"][0] == pytest.approx(p_small * math.sqrt(2), rel=1e-12)
+                # one kept and one dropped key: the single-gap bound is exact
+                assert r["gap_bound"][0] == pytest.approx(p_small, rel=1e-12)
             else:
                 assert r["k"][0] == 2 and r["tv"][0] == 0.0 and r["err"][0] == 0.0
+
+
+def test_single_gap_bound_exact_for_two_logit_levels():
+    """k keys at logit a and n - k at logit b < a: TV(k) = (n-k) e^b / (k e^a + (n-k) e^b)
+    = 1 / (1 + k/(n-k) e^(a-b)), which is the single-gap bound itself."""
+    d = 16
+    for n, k, gap in ((10, 3, 1.5), (50, 7, 3.0), (9, 1, 0.25)):
+        q = np.zeros((1, 1, 1, d), np.float32)
+        q[0, 0, 0, 0] = 4.0
+        K = np.zeros((1, 1, n, d), np.float32)
+        hi = np.random.default_rng(n).choice(n, size=k, replace=False)
+        K[0, 0, hi, 0] = gap  # scaled logit gap: 4 * gap / sqrt(16) = gap
+        V = np.random.default_rng(k).standard_normal((1, 1, n, d)).astype(np.float32)
+        tv_k = 1.0 / (1.0 + k / (n - k) * math.exp(gap))
+        tv_km1 = ((n - k) + math.exp(gap)) / (k * math.exp(gap) + (n - k))  # k - 1 of the top kept
+        eps = tv_k + 0.25 * (tv_km1 - tv_k)
+        r = oracle.certified_topk_attn(q, K, V, eps, n_heads=1, n_kv_heads=1)
+        assert r["k"][0] == k and r["idx"][0].tolist() == sorted(hi.tolist())
+        assert r["tv"][0] == pytest.approx(tv_k, rel=1e-12)
+        assert r["gap_bound"][0] == pytest.approx(tv_k, rel=1e-12)
 
 
 def test_gqa_head_mapping():
