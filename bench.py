@@ -352,7 +352,7 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": seconds * 1e3 / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {
             "workload": (f"{args.workload}: batch {prob.batch}, {prob.n_heads} query heads, "

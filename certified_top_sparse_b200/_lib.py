@@ -205,7 +205,9 @@ def cta_certified_topk_attn_noalloc(q, K, V, eps, *, out, k_out, idx_out, tv_out
                                     kl_out=None, status_dev=None, stream=None):
     """The no-allocation entry point: the library's own fixed scratch replaces
     the workspace.  Every output must be passed in (this wrapper allocates
-    nothing either).  See include/cta.h for its limits and ordering rules."""
+    nothing either).  Returns the same dict of (the caller's) tensors as
+    cta_certified_topk_attn.  See include/cta.h for its limits and ordering
+    rules."""
     batch, n_heads, m, d, n_kv_heads, n = _shape(q, K, V)
     o = make_opts(batch=batch, m=m, dtype=_dtype_code(q), stream=_stream_handle(stream),
                   err_out=err_out, kl_out=kl_out, status_dev=status_dev)
@@ -214,3 +216,4 @@ def cta_certified_topk_attn_noalloc(q, K, V, eps, *, out, k_out, idx_out, tv_out
                                                 _ptr(idx_out), _ptr(tv_out), ctypes.byref(o))
     if rc != CTA_OK:
         raise CtaError(rc, "cta_certified_topk_attn_noalloc")
+    return {"out": out, "k": k_out, "idx": idx_out, "tv": tv_out, "err": err_out, "kl": kl_out}

@@ -11,7 +11,7 @@
 namespace cta {
 namespace {
 
-constexpr int kTargetCtas = 148 * 6;   // ~6 resident CTAs per SM over 148 SMs
+constexpr int kCtasPerSmTarget = 6;    // score pass: ~6 resident CTAs per SM
 constexpr int64_t kMaxN = (int64_t)1 << 28;
 constexpr int kMaxChunks = 65535;      // grid.y limit
 
@@ -35,10 +35,10 @@ struct Layout {
 
 // Output pass: each CTA owns a contiguous range of chunks of one (group, row
 // tile); ranges are cut so that the ranges of all units about fill ctas_per_sm
-// CTAs on every SM.
-void set_ranges(Plan* p, int ctas_per_sm) {
+// CTAs on every one of the device's `sms` SMs.
+void set_ranges(Plan* p, int ctas_per_sm, int sms) {
   const int64_t units_out = (int64_t)p->groups * p->tiles_out;
-  int64_t nr = ((int64_t)ctas_per_sm * 148 + units_out - 1) / units_out;
+  int64_t nr = ((int64_t)ctas_per_sm * sms + units_out - 1) / units_out;
   if (nr > p->nchunks) nr = p->nchunks;
   if (nr < 1) nr = 1;
   p->range_len = (int)((p->nchunks + nr - 1) / nr);
@@ -46,7 +46,7 @@ void set_ranges(Plan* p, int ctas_per_sm) {
 }
 
 int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, int dtype,
-              double eps, Plan* p) {
+              double eps, int sms, Plan* p) {
   if (d != 64 && d != 128) return CTA_ERR_SHAPE;
   if (n < 1 || n > kMaxN) return CTA_ERR_SHAPE;
   if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0) return CTA_ERR_SHAPE;
@@ -72,7 +72,8 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   // Chunk: enough CTAs to fill the GPU, a multiple of 256 keys, at most 4096
   // keys (the logits of a tile are staged in shared memory).
   const int64_t units = groups * p->tiles_score;
-  const int64_t want = (kTargetCtas + units - 1) / units;
+  const int64_t target_ctas = (int64_t)kCtasPerSmTarget * sms;
+  const int64_t want = (target_ctas + units - 1) / units;
   int64_t chunk = (n + want - 1) / want;
   chunk = ((chunk + 255) / 256) * 256;
   if (chunk < 256) chunk = 256;
@@ -92,9 +93,9 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   // Selection: split rows over a cluster of up to 8 CTAs until ~2 CTAs per SM
   // are busy, keeping at least 4096 keys per CTA.
   int cs = 1;
-  while (cs < 8 && rows * cs * 2 <= 2 * 148 && n / (cs * 2) >= 4096) cs *= 2;
+  while (cs < 8 && rows * cs * 2 <= 2 * (int64_t)sms && n / (cs * 2) >= 4096) cs *= 2;
   p->sel_cluster = cs;
-  set_ranges(p, 2);
+  set_ranges(p, 2, sms);
   p->gparts = (p->n <= (int64_t)kShortMaxN) ? 1 : p->sel_cluster;
   return CTA_OK;
 }
@@ -154,7 +155,8 @@ size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const c
   cta_opts_init(&def);
   if (!o) o = &def;
   Plan p;
-  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, o->dtype, 0.5, &p) != CTA_OK) return 0;
+  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, o->dtype, 0.5, sm_count(), &p) != CTA_OK)
+    return 0;
   return layout(p).total;
 }
 
@@ -167,16 +169,17 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
   if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return CTA_ERR_ARG;
   Plan p;
-  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps, &p);
+  const int sms = sm_count();
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps, sms, &p);
   if (rc != CTA_OK) return rc;
   p.want_err = opts->err_out != nullptr;
-  set_ranges(&p, gather_ctas_per_sm(p.want_err));
+  set_ranges(&p, gather_ctas_per_sm(p.want_err), sms);
   // all-query tiles on the tensor cores: logits and value sums per 128-row tile
   const bool tc = score_tc_applies(p, opts->dtype);
   // decode-shaped bf16 value sums on the tensor cores
   const bool gtc = !tc && gather_tc_applies(p, opts->dtype);
   if (gtc) {
-    set_ranges_tc(&p, sm_count());
+    set_ranges_tc(&p, sms);
     p.nmax = p.nranges;  // the tensor-core logits pass writes one maximum per range
   }
   const Layout L = layout(p);
@@ -238,7 +241,8 @@ int cta_dense_attn(const void* q, const void* K, const void* V, int64_t n, int d
   if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
   if (!aligned16(q) || !aligned16(K) || !aligned16(V)) return CTA_ERR_ARG;
   Plan p;
-  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, 0.5, &p);
+  const int rc =
+      make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, 0.5, sm_count(), &p);
   if (rc != CTA_OK) return rc;
   if (launch_dense(opts->dtype, q, K, V, out, n, d, p.rows, p.gm,
                    static_cast<cudaStream_t>(opts->stream)) != cudaSuccess)

@@ -89,6 +89,7 @@ struct SelShared {
   unsigned int n_in;
   unsigned int rcount[kMaxCluster + 1];  // CTA 0: candidate counts per rank, then prefix
   int b1, b2, pos;
+  int row_shift;                    // fixed-point scale 2^row_shift of this row's exact masses
   float fbuf[kSelWarps];
 };
 
@@ -313,7 +314,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   const bool local_cc = (c1 - c0) <= kLocalChunks;
   uint32_t* cc = chunk_off + row * p.nchunks;
   const bool vec = (n & 3) == 0;
-  const float s2 = p.scale2, two_s = p.two_s;
+  const float s2 = p.scale2;
   const uint32_t chunk = (uint32_t)p.chunk;
 
   // The output pass counts finished ranges per (KV group, row tile): zeroed
@@ -388,6 +389,16 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
     unsigned long long sc[3] = {lsum, hsum, csum}, tot[3];
     block_scan_excl3(sc, tot, S);
     const unsigned long long ZL = tot[0], ZU = tot[1];
+    // The exact masses below use the scale 2^row_shift with Z * 2^row_shift
+    // <= 2^62: every sum fits 64 bits and the rounding of the n weights moves
+    // the total by at most n * 2^-(row_shift + 1) <= n * 2^-62 * Z_upper, a
+    // relative error of at most n * 2^-61 (<= 2^-33 for n <= 2^28), whatever
+    // the spread of the weights.  (One scale for every row, fixed by n alone,
+    // would lose up to n^2 * 2^-63 of the mass.)
+    if (tid == 0) {
+      const int e = ilogb((double)ZU * ldexp(1.0, -p.mass_shift)) + 1;  // Z_upper < 2^e
+      S.row_shift = min(62, 62 - max(e, 0));
+    }
     unsigned long long CL = sc[0], CU = sc[1], CN = sc[2];
     const double e_hi = p.eps * (1.0 - kDecideSlack), e_lo = p.eps * (1.0 + kDecideSlack);
     unsigned long long cn_before[kBinsPerThread];
@@ -418,6 +429,7 @@ select_kernel(const float* __restrict__ u, const float* __restrict__ cmax, RowSe
   const int b1 = min(S.b1, b2);
   unsigned long long n_above = S.n_above;
   unsigned long long n_in = S.n_in_s - n_above;
+  const float two_s = ldexpf(1.0f, S.row_shift);
   const bool direct = n_in <= (unsigned long long)kCap;
 
   // ---- 3. exact masses, candidates, certainly-kept counts per chunk -----------

@@ -59,6 +59,9 @@ def _load():
         ]
         lib.ora_dense_attn.restype = ctypes.c_int
         lib.ora_dense_attn.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, i64, i64, vp]
+        lib.ora_eval_kept_set.restype = ctypes.c_int
+        lib.ora_eval_kept_set.argtypes = [vp, vp, vp, ctypes.c_int, i64, i64, i64, i64, i64, i64,
+                                          vp, vp, vp, vp]
         assert lib.ora_nstat() == len(STAT_NAMES)
         _lib = lib
     return _lib
@@ -123,3 +126,34 @@ def dense_attn(q, K, V, *, n_heads, n_kv_heads, dtype=F32, batch=1, m=1):
     if rc != 0:
         raise RuntimeError(f"oracle dense attention failed with status {rc}")
     return out
+
+
+def eval_kept_set(q, K, V, sets, *, n_heads, n_kv_heads, dtype=F32, batch=1, m=1):
+    """The truncation to given kept sets, in fp64 (see ora_eval_kept_set).
+
+    ``sets`` is a list of one index array per row (distinct key indices, any
+    order, at least one).  Returns a dict with ``tv``, ``kl``, ``err``,
+    ``tv_drop_lowest`` (TV after removing the set's lowest-ranked key) [rows]
+    and ``out`` [rows, d].
+    """
+    lib = _load()
+    q, K, V = _raw(q, dtype), _raw(K, dtype), _raw(V, dtype)
+    d = q.shape[-1]
+    n = K.shape[-2]
+    rows = batch * n_heads * m
+    assert len(sets) == rows
+    packed = np.full((rows, n), -1, np.int32)
+    counts = np.zeros(rows, np.int32)
+    for r, s in enumerate(sets):
+        s = np.asarray(s, np.int64)
+        packed[r, : len(s)] = s
+        counts[r] = len(s)
+    out = np.zeros((rows, d), np.float64)
+    res = np.zeros((rows, 4), np.float64)
+    rc = lib.ora_eval_kept_set(q.ctypes.data, K.ctypes.data, V.ctypes.data, dtype, batch, n_heads,
+                               n_kv_heads, m, n, d, packed.ctypes.data, counts.ctypes.data,
+                               out.ctypes.data, res.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle set evaluation failed with status {rc}")
+    return {"tv": res[:, 0].copy(), "kl": res[:, 1].copy(), "err": res[:, 2].copy(),
+            "tv_drop_lowest": res[:, 3].copy(), "out": out}

@@ -20,7 +20,7 @@
  *   - refinements in terms of Var_P(V).
  * The logits are s_i = q.k_i / sqrt(d) (scaled dot-product attention).
  *
- * Readings where the page is silent (each is listed in the design doc):
+ * Readings where the page is silent:
  *   - ties in the logits are broken by the lower key index ranking first;
  *   - the ranking uses the exact fp64 dot product u_i = q.k_i (the scale
  *     1/sqrt(d) is positive, so the order is the same as for s_i, and ranking
@@ -454,4 +454,104 @@ int ora_dense_attn(const void* q, const void* K, const void* V, int dtype, int64
   }
   free(s);
   return 0;
+}
+
+/*
+ * The truncation to a GIVEN kept set, in fp64: the same definitions as above
+ * (abstract of "A Mathematical Theory of Top-k Sparse Attention via Total
+ * Variation Distance") applied to an arbitrary set S instead of the top k.
+ * Used to judge a kept set found elsewhere (for example by fp32 arithmetic
+ * near a boundary): P-hat = P restricted to S and renormalised, TV = sum of P
+ * over the keys outside S, out = mu_head = sum_S P_i v_i / sum_S P_i,
+ * err = TV ||mu_tail - mu_head||_2 with the tail the complement of S,
+ * KL(P-hat || P) from explicit log-probabilities, and the TV after dropping
+ * the lowest-ranked key of S (rank: logit descending, lower index first).
+ *
+ * sets [rows, n]: the first counts[row] entries of each row are the distinct
+ * key indices of S (any order), counts[row] >= 1.
+ * res [rows, 4]: TV(S), KL, err, TV(S minus its lowest-ranked key).
+ * out [rows, d].  Returns 0, -1 on bad arguments, -3 on allocation failure,
+ * -5 on a non-finite logit.
+ */
+int ora_eval_kept_set(const void* q, const void* K, const void* V, int dtype, int64_t batch,
+                      int64_t n_heads, int64_t n_kv_heads, int64_t m, int64_t n, int64_t d,
+                      const int32_t* sets, const int32_t* counts, double* out, double* res) {
+  if (!q || !K || !V || !sets || !counts || !out || !res) return -1;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0 || n < 1 || d < 1 || m < 1 ||
+      batch < 1)
+    return -1;
+  const int64_t group = n_heads / n_kv_heads;
+  const int64_t rows = batch * n_heads * m;
+  double* u = (double*)malloc(sizeof(double) * (size_t)n);
+  double* w = (double*)malloc(sizeof(double) * (size_t)n);
+  unsigned char* in_s = (unsigned char*)malloc((size_t)n);
+  csum* acc = (csum*)malloc(sizeof(csum) * 2 * (size_t)d);
+  if (!u || !w || !in_s || !acc) {
+    free(u); free(w); free(in_s); free(acc);
+    return -3;
+  }
+  const double inv_sqrt_d = 1.0 / sqrt((double)d);
+  int status = 0;
+  for (int64_t row = 0; row < rows && status == 0; ++row) {
+    const int64_t bh = row / m;
+    const int64_t h = bh % n_heads, b = bh / n_heads;
+    const int64_t kv_base = (b * n_kv_heads + h / group) * n * d;
+    const int64_t cnt = counts[row];
+    if (cnt < 1 || cnt > n) { status = -1; break; }
+    /* logits and the row maximum */
+    double mx = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+      double x = 0.0;
+      for (int64_t t = 0; t < d; ++t)
+        x += widen(q, dtype, row * d + t) * widen(K, dtype, kv_base + i * d + t);
+      if (!isfinite(x)) { status = -5; break; }
+      u[i] = x;
+      if (x > mx) mx = x;
+    }
+    if (status != 0) break;
+    memset(in_s, 0, (size_t)n);
+    int64_t low = -1;  /* lowest-ranked key of S */
+    for (int64_t r = 0; r < cnt; ++r) {
+      const int64_t i = sets[row * n + r];
+      if (i < 0 || i >= n || in_s[i]) { status = -1; break; }
+      in_s[i] = 1;
+      if (low < 0 || u[i] < u[low] || (u[i] == u[low] && i > low)) low = i;
+    }
+    if (status != 0) break;
+    /* masses: kept, dropped, total; sums in key index order */
+    csum zs = {0.0, 0.0}, hs = {0.0, 0.0}, ts = {0.0, 0.0};
+    for (int64_t t = 0; t < 2 * d; ++t) { acc[t].s = 0.0; acc[t].c = 0.0; }
+    for (int64_t i = 0; i < n; ++i) {
+      w[i] = exp((u[i] - mx) * inv_sqrt_d);
+      cs_add(&zs, w[i]);
+      cs_add(in_s[i] ? &hs : &ts, w[i]);
+      csum* a = acc + (in_s[i] ? 0 : d);
+      for (int64_t t = 0; t < d; ++t) cs_add(&a[t], w[i] * widen(V, dtype, kv_base + i * d + t));
+    }
+    const double Z = cs_val(&zs), Hm = cs_val(&hs), Tm = cs_val(&ts);
+    const double logZ = log(Z), logH = log(Hm);
+    csum kl = {0.0, 0.0};
+    for (int64_t i = 0; i < n; ++i) {
+      if (!in_s[i]) continue;
+      const double s_rel = (u[i] - mx) * inv_sqrt_d;
+      const double phat = w[i] / Hm;
+      cs_add(&kl, phat * ((s_rel - logH) - (s_rel - logZ)));
+    }
+    double e2 = 0.0;
+    for (int64_t t = 0; t < d; ++t) {
+      const double mu_h = cs_val(&acc[t]) / Hm;
+      out[row * d + t] = mu_h;
+      if (Tm > 0.0) {
+        const double mu_t = cs_val(&acc[d + t]) / Tm;
+        e2 += (mu_t - mu_h) * (mu_t - mu_h);
+      }
+    }
+    const double tv = Tm / Z;
+    res[row * 4 + 0] = tv;
+    res[row * 4 + 1] = cs_val(&kl);
+    res[row * 4 + 2] = (Tm > 0.0) ? tv * sqrt(e2) : 0.0;
+    res[row * 4 + 3] = (Tm + w[low]) / Z;
+  }
+  free(u); free(w); free(in_s); free(acc);
+  return status;
 }

@@ -39,12 +39,15 @@ def test_library_exports_every_declared_symbol():
         assert re.search(rf"\bT {name}$", out, re.M), name
 
 
-def test_library_targets_sm100a():
-    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", cta.LIB_PATH],
-                         capture_output=True, text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    assert "sm_100a" in out.stdout
+def test_library_is_built_for_sm100a_only():
+    """The build compiles one cubin for sm_100a and embeds no PTX, so a launch
+    on any other architecture fails instead of JIT-compiling something else;
+    every GPU test then exercises exactly this code (checked from the build
+    recipe, without inspecting the binary)."""
+    from certified_top_sparse_b200 import build as cta_build
+    flags = " ".join(cta_build.FLAGS)
+    assert "-gencode arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1 and "code=compute_" not in flags
 
 
 def test_version_and_strings():

@@ -294,3 +294,89 @@ def test_gqa_head_mapping():
     k1 = r["k"].reshape(2, 8)
     k2 = r2["k"].reshape(2, 8)
     np.testing.assert_array_equal(k2, k1[:, qperm])
+
+
+# ---------------------------------------------------------------------------
+# the truncation to a given kept set, and the fp32 tie allowance
+
+KEPT = os.path.join(os.path.dirname(__file__), "golden", "kept_set_and_tie_bound.json")
+
+
+def _ev2(expr: str) -> float:
+    return float(eval(expr.replace("^", "**"), {"__builtins__": {}},
+                      {"ln": math.log, "sqrt": math.sqrt, "exp": math.exp}))
+
+
+def test_eval_kept_set_hand_derived():
+    """Arbitrary (non-top-k) kept sets of the four-key example, hand-derived."""
+    c = json.load(open(KEPT))["kept_set_cases"]
+    d = c["d"]
+    q = np.array(c["q"], np.float32).reshape(1, 1, 1, d)
+    K = np.array(c["K"], np.float32).reshape(1, 1, -1, d)
+    V = np.array(c["V"], np.float32).reshape(1, 1, -1, d)
+    for s in c["sets"]:
+        r = oracle.eval_kept_set(q, K, V, [s["set"]], n_heads=1, n_kv_heads=1)
+        for key in ("tv", "kl", "err", "tv_drop_lowest"):
+            assert r[key][0] == pytest.approx(_ev2(s[key]), abs=1e-7), (s["set"], key)
+        np.testing.assert_allclose(r["out"][0], [_ev2(x) for x in s["out"]], atol=1e-7)
+
+
+@pytest.mark.parametrize("prob", list(_small_problems()), ids=lambda p: p.name)
+def test_eval_kept_set_on_the_top_k_set(prob):
+    """On the certified set itself the set evaluation reproduces the main
+    routine's TV, KL, err and output, and dropping the lowest kept key gives
+    TV(k - 1); on a perturbed set (the last kept key swapped for the first
+    dropped one) TV grows by exactly their mass difference."""
+    o = _run(prob)
+    dt = oracle.BF16 if str(prob.q.dtype) == "torch.bfloat16" else oracle.F32
+    raw = dict(n_heads=prob.n_heads, n_kv_heads=prob.n_kv_heads, dtype=dt, batch=prob.batch,
+               m=prob.m)
+    e = oracle.eval_kept_set(W.raw_words(prob.q), W.raw_words(prob.K), W.raw_words(prob.V),
+                             o["idx"], **raw)
+    np.testing.assert_allclose(e["tv"], o["tv"], rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(e["kl"], o["kl"], rtol=1e-9, atol=1e-14)
+    np.testing.assert_allclose(e["err"], o["err"], rtol=1e-9, atol=1e-14)
+    np.testing.assert_allclose(e["out"], o["out"], rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(e["tv_drop_lowest"], o["tv_km1"], rtol=1e-10, atol=1e-14)
+
+
+def test_eval_kept_set_brute_force_masses():
+    """TV of random subsets of a tiny row equals the dropped mass of an
+    independent numpy softmax (fp64 from the same fp32 inputs)."""
+    rng = np.random.default_rng(5)
+    n, d = 11, 8
+    q = rng.standard_normal((1, 1, 1, d)).astype(np.float32) * 2
+    K = rng.standard_normal((1, 1, n, d)).astype(np.float32)
+    V = rng.standard_normal((1, 1, n, d)).astype(np.float32)
+    u = K[0, 0].astype(np.float64) @ q[0, 0, 0].astype(np.float64)
+    P = np.exp((u - u.max()) / math.sqrt(d))
+    P /= P.sum()
+    order = sorted(range(n), key=lambda i: (-u[i], i))
+    for trial in range(40):
+        size = int(rng.integers(1, n + 1))
+        s = rng.choice(n, size, replace=False)
+        r = oracle.eval_kept_set(q, K, V, [s], n_heads=1, n_kv_heads=1)
+        keep = np.zeros(n, bool)
+        keep[s] = True
+        assert r["tv"][0] == pytest.approx(P[~keep].sum(), abs=1e-13)
+        low = max(s, key=lambda i: order.index(i))
+        assert r["tv_drop_lowest"][0] == pytest.approx(P[~keep].sum() + P[low], abs=1e-13)
+        mu = (P[keep, None] * V[0, 0][keep].astype(np.float64)).sum(0) / P[keep].sum()
+        np.testing.assert_allclose(r["out"][0], mu, rtol=1e-12, atol=1e-13)
+
+
+def test_tie_bound_hand_derived():
+    """The fp32 rounding allowance of the boundary keys (class T of the parity
+    tests): gamma_d with 2^-24 and absolute products of both boundary keys."""
+    c = json.load(open(KEPT))["tie_bound_case"]
+    d = c["d"]
+    q = np.array(c["q"], np.float32).reshape(1, 1, 1, d)
+    K = np.array(c["K"], np.float32).reshape(1, 1, -1, d)
+    V = np.zeros_like(K)
+    r = oracle.certified_topk_attn(q, K, V, c["eps"], n_heads=1, n_kv_heads=1)
+    e = c["expect"]
+    assert int(r["k"][0]) == e["k"] and r["idx"][0].tolist() == e["idx"]
+    assert r["gap_u"][0] == _ev2(e["gap_u"])
+    assert r["tie_bound"][0] == pytest.approx(_ev2(e["tie_bound"]), rel=1e-15)
+    assert r["tv"][0] == pytest.approx(_ev2(e["tv"]), rel=1e-12)
+    assert r["gap_bound"][0] == pytest.approx(_ev2(e["gap_bound"]), rel=1e-12)
