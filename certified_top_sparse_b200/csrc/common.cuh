@@ -37,7 +37,9 @@ struct Plan {
   int rstages;          // tensor-core output pass: 128-key stages per range (0: not used)
   int nmax;             // partial row maxima per row in cmax (per chunk, or per range of
                         // the tensor-core logits pass); row stride nchunks
+  int settle_group;     // tensor-core decode path: value-pass ranges per CTA of the last kernel
 };
+
 
 // Per-row result of the selection pass.
 struct RowSel {
@@ -105,6 +107,126 @@ __device__ __forceinline__ unsigned long long fixed_mass(float w, float two_s) {
 __device__ __forceinline__ bool certified(unsigned long long Z, unsigned long long C, double eps) {
   return (double)(Z - C) / (double)Z <= eps;
 }
+
+// ---------------------------------------------------------------------------
+// Tensor-core decode path: exact masses in 128-bit fixed point, key levels and
+// the records the three kernels of that path exchange through the workspace.
+
+// Unsigned 128-bit integer (two 64-bit words) for exact mass sums: every
+// weight w in [0, 1] becomes round(w * 2^62), so any number of them adds up
+// without overflow and without depending on the order of the additions.
+struct U128 {
+  unsigned long long lo, hi;
+};
+constexpr int kMass62 = 62;
+__device__ __forceinline__ U128 u128_zero() { return U128{0ull, 0ull}; }
+__device__ __forceinline__ void u128_add(U128& a, unsigned long long x) {
+  asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, 0;" : "+l"(a.lo), "+l"(a.hi) : "l"(x));
+}
+__device__ __forceinline__ void u128_add(U128& a, const U128& b) {
+  asm("add.cc.u64 %0, %0, %2;\n\taddc.u64 %1, %1, %3;" : "+l"(a.lo), "+l"(a.hi) : "l"(b.lo), "l"(b.hi));
+}
+__device__ __forceinline__ U128 u128_sub(U128 a, const U128& b) {
+  asm("sub.cc.u64 %0, %0, %2;\n\tsubc.u64 %1, %1, %3;" : "+l"(a.lo), "+l"(a.hi) : "l"(b.lo), "l"(b.hi));
+  return a;
+}
+__device__ __forceinline__ bool u128_lt(const U128& a, const U128& b) {
+  return a.hi < b.hi || (a.hi == b.hi && a.lo < b.lo);
+}
+__device__ __forceinline__ double u128_to_double(const U128& a) {
+  return (double)a.hi * 18446744073709551616.0 + (double)a.lo;
+}
+// Sum over the 32 lanes of a warp (butterfly: every lane ends with the total).
+__device__ __forceinline__ U128 u128_warp_sum(U128 a) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    U128 b;
+    b.lo = __shfl_xor_sync(0xffffffffu, a.lo, o);
+    b.hi = __shfl_xor_sync(0xffffffffu, a.hi, o);
+    u128_add(a, b);
+  }
+  return a;
+}
+// The weight w (fp32, 0 <= w <= 1) in units of 2^-62.
+__device__ __forceinline__ unsigned long long mass62(float w) {
+  return __float2ull_rn(__fmul_rn(fmaxf(w, 0.0f), 4.611686018427387904e18f));
+}
+// The certificate test on exact masses: (Z - C) / Z <= eps, in fp64.
+__device__ __forceinline__ bool certified128(const U128& Z, const U128& C, double eps) {
+  return u128_to_double(u128_sub(Z, C)) / u128_to_double(Z) <= eps;
+}
+
+// Level of a logit: ceil(64 x) with x = u * log2(e)/sqrt(d) rounded to fp32,
+// i.e. the key's position on a grid of 1/64 of a halving of the weight.  It is
+// a non-decreasing function of u, so a level interval is an interval of the
+// ranking; every kernel computes it with these exact operations.  NaN and
+// huge values are clamped (their rows are flagged non-finite).
+constexpr int kLevelsPerOctave = 64;
+__device__ __forceinline__ int key_level(float u, float scale2) {
+  float x = __fmul_rn(u, scale2);
+  x = fminf(fmaxf(x, -1.0e6f), 1.0e6f);
+  return __float2int_ru(x * (float)kLevelsPerOctave);
+}
+
+// Per (row, key range) level histogram written by the tensor-core logits pass.
+// Fine bin i counts the range's keys of level top - i; octave o of the frame
+// is bins 64 o .. 64 o + 63.  top is a multiple of 64 set from the range's
+// first stage (its largest level rounded up, plus kHistHeadroom octaves).
+constexpr int kHistOctaves = 48;
+constexpr int kHistHeadroom = 16;                        // octaves above the first stage's max
+constexpr int kHistBins = kHistOctaves * kLevelsPerOctave;  // 3072
+constexpr uint32_t kHistAbove = 0x1u;   // a key lay above the frame: the record is unusable
+constexpr uint32_t kHistSaturated = 0x2u;  // a fine count exceeded 65535
+struct RangeHist {
+  int32_t top;                  // level of fine bin 0 (multiple of 64)
+  uint32_t flags;               // kHistAbove | kHistSaturated
+  uint32_t below;               // keys below the frame (level <= top - kHistBins)
+  uint32_t pad;
+  uint32_t ocnt[kHistOctaves];  // keys per octave
+  float omass[kHistOctaves];    // per octave: sum over its bins j of count * 2^(-j/64)
+  uint16_t fine[kHistBins];     // keys per fine bin (saturating)
+};
+static_assert(sizeof(RangeHist) % 16 == 0, "records are read with 16-byte loads");
+
+// Per row: the level bracket of the cut that the value pass used.  Keys with
+// level >= lhi are kept for certain, keys with level < llo dropped for certain,
+// the window llo <= level < lhi is settled once the exact cut is known.
+struct RowBracket {
+  float M;        // largest logit of the row
+  int32_t llo, lhi;
+  uint32_t pad;
+};
+
+// Per (row, key range): what the value pass accumulated over the range's keys.
+struct RangeRec {
+  U128 mh, mt, mw;   // exact masses (2^-62 units) of the kept, dropped and window keys
+  double wh, wt;     // weight sums of the kept and dropped keys (window keys excluded),
+                     // fp32 per stage and lane, fp64 above: an independent reduction for KL
+  uint32_t nh, nw;   // kept and window key counts
+  float tmax;        // largest logit among the dropped keys (-inf if none)
+  uint32_t pad;
+};
+static_assert(sizeof(RangeRec) % 16 == 0, "16-byte records");
+
+// Per (row, key range) after the last kernel has settled the range's window keys.
+struct SegRec {
+  double wh, wt;     // weight sums (for KL) of the kept and dropped keys of the range
+  float tmax;        // largest dropped logit of the range
+  uint32_t pad[3];
+};
+
+constexpr int kCandCap = 2048;   // window keys per row kept as candidates for the exact cut
+
+// Workspace regions of the tensor-core decode path (device pointers, set per call).
+struct TcBufs {
+  RangeHist* hist;       // [rows][nranges]
+  RangeRec* rrec;        // [rows][nranges]
+  SegRec* srec;          // [rows][nranges]
+  RowBracket* brk;       // [rows]
+  unsigned long long* cand;  // [rows][kCandCap] composite keys of window keys
+  uint32_t* cand_cnt;    // [rows] window keys seen (zeroed by the logits pass)
+  uint32_t* ticket;      // [rows] ranges settled (zeroed by the logits pass)
+};
 
 // ---------------------------------------------------------------------------
 // 16-byte streaming load (read-only path, no L1 allocation).

@@ -30,7 +30,10 @@ int ceil_log2(int64_t n) {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t u, cmax, sel, choff, acc, gmax, unit, status, total;
+  size_t u, cmax, sel, choff, acc, gmax, unit, status;
+  // tensor-core decode path only (zero-sized otherwise)
+  size_t hist, rrec, srec, brk, cand, cand_cnt, ticket;
+  size_t total;
 };
 
 // Output pass: each CTA owns a contiguous range of chunks of one (group, row
@@ -100,7 +103,7 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   return CTA_OK;
 }
 
-Layout layout(const Plan& p) {
+Layout layout(const Plan& p, bool tc_decode) {
   Layout L;
   size_t off = 0;
   L.u = off;      off = align256(off + sizeof(float) * (size_t)p.rows * (size_t)p.ustride);
@@ -111,8 +114,48 @@ Layout layout(const Plan& p) {
   L.gmax = off;   off = align256(off + sizeof(float) * (size_t)p.rows * kMaxGParts);
   L.unit = off;   off = align256(off + sizeof(uint32_t) * (size_t)p.rows);
   L.status = off; off = align256(off + sizeof(uint32_t));
+  const size_t rr = tc_decode ? (size_t)p.rows * p.nranges : 0;
+  const size_t rw = tc_decode ? (size_t)p.rows : 0;
+  L.hist = off;     off = align256(off + sizeof(RangeHist) * rr);
+  L.rrec = off;     off = align256(off + sizeof(RangeRec) * rr);
+  L.srec = off;     off = align256(off + sizeof(SegRec) * rr);
+  L.brk = off;      off = align256(off + sizeof(RowBracket) * rw);
+  L.cand = off;     off = align256(off + sizeof(unsigned long long) * kCandCap * rw);
+  L.cand_cnt = off; off = align256(off + sizeof(uint32_t) * rw);
+  L.ticket = off;   off = align256(off + sizeof(uint32_t) * rw);
   L.total = off;
   return L;
+}
+
+// The complete launch plan of one call: shapes, chunking, which kernels run
+// (all-query tensor-core tiles, the tensor-core decode path, or the CUDA-core
+// kernels) and their ranges.  Used by cta_workspace_size and the call itself.
+struct CallPlan {
+  Plan p;
+  bool tc;   // all-query tensor-core tiles
+  bool gtc;  // tensor-core decode path
+};
+
+int plan_call(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, int dtype,
+              double eps, bool want_err, CallPlan* cp) {
+  const int sms = sm_count();
+  const int rc = make_plan(n, d, n_heads, n_kv_heads, batch, m, dtype, eps, sms, &cp->p);
+  if (rc != CTA_OK) return rc;
+  Plan& p = cp->p;
+  p.want_err = want_err ? 1 : 0;
+  set_ranges(&p, gather_ctas_per_sm(want_err), sms);
+  cp->tc = score_tc_applies(p, dtype);
+  cp->gtc = !cp->tc && gather_tc_applies(p, dtype);
+  if (cp->gtc) {
+    set_ranges_tc(&p, sms);
+    p.nmax = p.nranges;  // the tensor-core logits pass writes one maximum per range
+    // the last kernel: the fewest value-pass ranges per CTA that let every CTA
+    // be resident at once (two per SM)
+    int g = 1;
+    while (g < 32 && (int64_t)p.rows * ((p.nranges + g - 1) / g) > 2 * (int64_t)sms) ++g;
+    p.settle_group = g;
+  }
+  return CTA_OK;
 }
 
 bool aligned16(const void* x) { return ((uintptr_t)x & 15u) == 0; }
@@ -154,10 +197,10 @@ size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const c
   cta_opts def;
   cta_opts_init(&def);
   if (!o) o = &def;
-  Plan p;
-  if (make_plan(n, d, n_heads, n_kv_heads, o->batch, o->m, o->dtype, 0.5, sm_count(), &p) != CTA_OK)
+  CallPlan cp;
+  if (plan_call(n, d, n_heads, n_kv_heads, o->batch, o->m, o->dtype, 0.5, true, &cp) != CTA_OK)
     return 0;
-  return layout(p).total;
+  return layout(cp.p, cp.gtc).total;
 }
 
 int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t n, int d,
@@ -168,21 +211,13 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   if (!opts) return CTA_ERR_WORKSPACE;  // the workspace is mandatory
   if (opts->dtype != CTA_F32 && opts->dtype != CTA_BF16) return CTA_ERR_ARG;
   if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return CTA_ERR_ARG;
-  Plan p;
-  const int sms = sm_count();
-  const int rc = make_plan(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps, sms, &p);
+  CallPlan cp;
+  const int rc = plan_call(n, d, n_heads, n_kv_heads, opts->batch, opts->m, opts->dtype, eps,
+                           opts->err_out != nullptr, &cp);
   if (rc != CTA_OK) return rc;
-  p.want_err = opts->err_out != nullptr;
-  set_ranges(&p, gather_ctas_per_sm(p.want_err), sms);
-  // all-query tiles on the tensor cores: logits and value sums per 128-row tile
-  const bool tc = score_tc_applies(p, opts->dtype);
-  // decode-shaped bf16 value sums on the tensor cores
-  const bool gtc = !tc && gather_tc_applies(p, opts->dtype);
-  if (gtc) {
-    set_ranges_tc(&p, sms);
-    p.nmax = p.nranges;  // the tensor-core logits pass writes one maximum per range
-  }
-  const Layout L = layout(p);
+  const Plan& p = cp.p;
+  const bool tc = cp.tc, gtc = cp.gtc;
+  const Layout L = layout(p, gtc);
   if (!opts->workspace || ((uintptr_t)opts->workspace & 255u) != 0 || opts->workspace_bytes < L.total)
     return CTA_ERR_WORKSPACE;
 
@@ -199,9 +234,30 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
   void** ev = opts->phase_events;
 
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
-  if ((tc    ? launch_score_tc(q, K, u, p, status, st)
-       : gtc ? launch_score_kv_tc(q, K, u, cmax, p, status, st)
-             : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) != cudaSuccess)
+  if (gtc) {
+    // tensor-core decode path: logits (+ level histograms), the bracketed
+    // value pass (+ exact masses), then the exact cut, indices and outputs
+    TcBufs tb;
+    tb.hist = reinterpret_cast<RangeHist*>(ws + L.hist);
+    tb.rrec = reinterpret_cast<RangeRec*>(ws + L.rrec);
+    tb.srec = reinterpret_cast<SegRec*>(ws + L.srec);
+    tb.brk = reinterpret_cast<RowBracket*>(ws + L.brk);
+    tb.cand = reinterpret_cast<unsigned long long*>(ws + L.cand);
+    tb.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cand_cnt);
+    tb.ticket = reinterpret_cast<uint32_t*>(ws + L.ticket);
+    if (launch_score_kv_tc(q, K, u, cmax, tb, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+    if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (launch_gather_tc(V, u, cmax, tb, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+    if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (launch_settle_tc(V, u, tb, acc, out, k_out, idx_out, tv_out, opts->err_out, opts->kl_out,
+                         opts->gap_out, p, status, st) != cudaSuccess)
+      return CTA_ERR_CUDA;
+    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;
+    return CTA_OK;
+  }
+  if ((tc ? launch_score_tc(q, K, u, p, status, st)
+          : launch_score(opts->dtype, q, K, u, cmax, p, status, st)) != cudaSuccess)
     return CTA_ERR_CUDA;
   if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
   if ((select_short_applies(p)
@@ -216,12 +272,6 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
                      st) != cudaSuccess)
       return CTA_ERR_CUDA;
     if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-  } else if (gtc) {  // tensor-core value sums, then the row-parallel finalisation
-    if (launch_gather_tc(V, u, sel, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
-    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
-    if (launch_finalize_tc(acc, sel, gmax, out, opts->err_out, opts->kl_out, opts->gap_out, p,
-                           status, st) != cudaSuccess)
-      return CTA_ERR_CUDA;
   } else {  // value sums, then the last CTA of each row tile finalises it
     if (launch_gather(opts->dtype, V, u, sel, acc, unit_cnt, gmax, out, opts->err_out,
                       opts->kl_out, opts->gap_out, p, status, st) != cudaSuccess)

@@ -1,46 +1,70 @@
-// Phases 3 and 4 for decode-shaped problems (bf16 values, d = 128) on the
-// 5th-generation tensor cores.
+// Phase 2-3 for decode-shaped problems (bf16 values, d = 128): the value pass
+// on the 5th-generation tensor cores, which needs only a bracket of the cut,
+// not the cut itself.
 //
 // Method ("A Mathematical Theory of Top-k Sparse Attention via Total Variation
-// Distance", arXiv 2512.07647, abstract): with the exact head-tail
-// decomposition Attn = H mu_head + tau mu_tail, the truncated output is mu_head
-// and the error needs mu_tail, i.e. per row the kept sum sum_{kept} w_i v_i
-// and the dropped sum sum_{dropped} w_i v_i over all n value rows.
+// Distance", arXiv 2512.07647, abstract): certified Top-k keeps the minimal
+// k_eps keys whose discarded softmax tail mass TV is <= eps; with the exact
+// head-tail decomposition Attn = H mu_head + tau mu_tail the truncated output
+// is mu_head and the error needs mu_tail, i.e. per row the kept sum
+// sum_{kept} w_i v_i and the dropped sum sum_{dropped} w_i v_i.
 //
-// For the (at most four) query rows of a row tile, which share one KV head,
-// these sums are one contraction per stage of 128 keys:
+// The bracket.  From the level histograms of the logits pass (RangeHist) the
+// weight warps bound, for every level boundary, the mass of the keys below it
+// from above and from below (a level is 1/64 of a halving of the weight, so
+// every key's weight is known within a factor 2^(1/64) from its level alone),
+// and the total mass likewise.  The cut lies where the mass below reaches eps
+// of the total, so every key whose level is certainly above that point is
+// kept (level >= lhi) and every key certainly below is dropped (level < llo);
+// the keys between (the window, typically a few hundred per row) are left to
+// the last kernel, which finds the exact cut among them.  Octave totals of the
+// histograms locate the octave(s) of the cut; only their fine bins are read.
+//
+// The value sums.  For the (at most four) query rows of a row tile, which
+// share one KV head, the kept and dropped sums are one contraction per stage
+// of 128 keys:
 //     S[dim][c] += sum_key V[key][dim] W[c][key],
 // column c running over (kept, dropped) x (three bf16 parts of the fp32
 // weight) x row.  The parts hi = bf16(w), mid = bf16(w - hi), lo = bf16(w -
 // hi - mid) carry the fp32 weight to about 2^-24 relative, and bf16 x bf16
-// products are exact in the fp32 accumulator, so the sums match fp32
-// multiply-adds up to the order of addition.  The CUDA cores only turn logits
-// into weights; value rows go from HBM to shared memory by TMA and from there
-// into tcgen05.mma as the MN-major A operand (M = 128 dimensions), the weights
-// are the K-major B operand (N = 32, unused columns zero), and the sums
-// accumulate in tensor memory over the whole key range of a work item.
+// products are exact in the fp32 accumulator.  Window keys get weight 0 in
+// both columns.  The value stages (V) come from HBM by TMA as the MN-major A
+// operand (M = 128 dimensions), the weights are the K-major B operand (N = 32,
+// unused columns zero), and the sums accumulate in tensor memory over the
+// whole key range of a work item.
+//
+// The exact masses.  Alongside, every key's weight becomes an integer in units
+// of 2^-62 (mass62) and is added, in 128 bits, to the kept, dropped or window
+// mass of its row and range: exact and order-independent, so the last kernel's
+// certificate test is exact too.  Window keys also go to a per-row candidate
+// list (composite key: logit order, then index).  Per range the pass writes a
+// RangeRec: the three masses, fp64 weight sums of the kept and dropped keys,
+// their counts and the largest dropped logit.
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0     TMA: each stage is two 64-dimension boxes of 128 keys (128-byte
-//              swizzle) into a ring of kGStages slots;
+//              swizzle) into a ring of kGStages slots, and the stage's logits
+//              of the tile's rows (bulk copies on a barrier of their own);
 //   warp 1     MMA: 8 MMAs (K = 16) per stage, whose commit frees the slot; at
 //              the end of an item a commit hands the accumulator over; owns
-//              the tensor memory (two accumulators, so an item's epilogue
-//              overlaps the next item's stream);
-//   warp 0     also brings the stage's logits of the tile's rows (bulk copies
-//              on the same barrier), so the weight warps read shared memory only;
-//   warps 2-5  weights: warp r writes row r's part of the stage's W tile;
+//              the tensor memory (two accumulators);
+//   warps 2-5  weights: warp r computes row r's bracket once per work item,
+//              then writes row r's part of each stage's W tile and its masses;
 //   warps 6-9  epilogue: read the accumulator, add the parts in fp64, write
 //              the range partial.
 // Work items are (KV group, key range, row tile) with ranges cut in stages so
-// that every SM gets about the same number of stages.  A second, row-parallel
-// kernel (one CTA per row, all range partials loaded at once) forms the
-// outputs; it is launched as a programmatic dependent so that its launch
-// overlaps the tail of this one.
+// that every SM gets about the same number of stages.
+//
+// Ordering: launched as a programmatic dependent of the logits pass.  Its CTAs
+// can start only after every logits CTA has passed its own wait for the
+// caller's preceding kernel, so the value rows may stream at once: the
+// producer fills the first ring of value stages before it waits for the
+// logits pass to complete (griddepcontrol.wait) and only then loads logits.
+// The weight warps wait likewise before they read the histograms.
 #include <algorithm>
+#include <climits>
 
 #include "common.cuh"
-#include "finalize.cuh"  // single_gap_bound
 #include "kernels.cuh"
 #include "umma.cuh"
 
@@ -63,9 +87,13 @@ constexpr int kGEpiWarp0 = 6;
 constexpr int kGEpiThreads = 4 * kWarp;
 constexpr int kGEpiBar = 1;           // named barrier of the epilogue warps
 constexpr uint32_t kGTmemCols = 2 * kGN;
-constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU);
+constexpr int kCandBuf = 256;         // window keys a weight warp buffers (>= 128: one stage's)
+constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU) + 4 * kCandBuf * 8;
 static_assert(kGK % 64 == 0 && kGK <= 256, "a stage is whole 64-key swizzle atoms, one TMA box");
 static_assert(kGSmem <= 227 * 1024, "shared memory");
+
+constexpr int kMergeOct = 64;         // octaves of the merged per-row frame (two per lane)
+constexpr int kFineOctMax = 4;        // window octaves refined with the fine counts
 
 struct GItem {
   int tile, range, group;
@@ -102,12 +130,281 @@ __device__ __forceinline__ bool aborted(const int* flag) {
   return *reinterpret_cast<const volatile int*>(flag) != 0;
 }
 
+// 2^e exactly, for -1022 <= e <= 1023 (0 below): built from the exponent bits.
+__device__ __forceinline__ double pow2i(int e) {
+  return e < -1022 ? 0.0 : __longlong_as_double((long long)(1023 + min(e, 1023)) << 52);
+}
+
+// Inclusive suffix sums across the lanes (lane l gets the sum over lanes >= l).
+__device__ __forceinline__ double warp_suffix_sum(double v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane + o < 32) v += y;
+  }
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Appends a warp's buffered window keys buf[0, nb) to the row's candidate list
+// (all are counted; keys beyond the list's capacity are dropped, which the
+// last kernel detects from the count).  Whole warp.
+__device__ __forceinline__ void flush_cands(const unsigned long long* buf, uint32_t nb,
+                                            unsigned long long* cand, uint32_t* cnt) {
+  const int lane = threadIdx.x & 31;
+  uint32_t base = 0u;
+  if (lane == 0) base = atomicAdd(cnt, nb);
+  base = __shfl_sync(0xffffffffu, base, 0);
+  for (uint32_t i = lane; i < nb; i += 32)
+    if (base + i < (uint32_t)kCandCap) cand[base + i] = buf[i];
+  __syncwarp();
+}
+
+// The bracket of one row's cut, computed by one warp from the row's range
+// histograms and range maxima.  Returns (llo, lhi) through the references and
+// the row maximum M.  Every CTA that handles a range of the row computes the
+// same values from the same data.
+//
+// Frame: T = 64 ceil(X_M), X_M = fl(M * scale2), so every key's level is <= T;
+// merged fine index g = T - level, octave O = g / 64.  A key with fine index g
+// has weight w = 2^-a with a within E of X_M - (T - g)/64 ... X_M - (T - g - 1)/64,
+// i.e. 2^(delta - (g + 1)/64) <= w <= 2^(delta - g/64) up to the relative slack
+// s, where delta = T/64 - X_M in [0, 1) and E covers the fp32 rounding of
+// a = (M - u) * scale2 against X_M - x, exp2f's error and the octave sums' own
+// fp32 rounding.
+__device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __restrict__ cmax,
+                            int64_t row, const Plan& p, float& M_out, int& llo, int& lhi) {
+  const int lane = threadIdx.x & 31;
+  const int nr = p.nranges;
+  const RangeHist* rh = hist + row * nr;
+  // Round 0 of the loads, all issued before any is used: the range maxima, the
+  // headers and the octave sums of ranges 0 .. 31 (octave o in lane o % 32).
+  int top0 = 0;
+  uint32_t flags0 = 0u, below0 = 0u;
+  float oa0[32], ob0[32];
+  const int nb0 = min(32, nr);
+  float M = kNegInf;
+  if (lane < nr) {
+    M = __ldcg(cmax + row * p.nchunks + lane);
+    top0 = __ldcg(&rh[lane].top);
+    flags0 = __ldcg(&rh[lane].flags);
+    below0 = __ldcg(&rh[lane].below);
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    oa0[j] = 0.0f;
+    ob0[j] = 0.0f;
+    if (j < nb0) {
+      oa0[j] = __ldcg(&rh[j].omass[lane]);
+      if (lane + 32 < kHistOctaves) ob0[j] = __ldcg(&rh[j].omass[lane + 32]);
+    }
+  }
+  for (int r = 32 + lane; r < nr; r += 32) M = fmaxf(M, __ldcg(cmax + row * p.nchunks + r));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  M_out = M;
+  llo = INT_MIN;  // defaults: every key is in the window
+  lhi = INT_MAX;
+  const float XM = __fmul_rn(M, p.scale2);
+  if (!(fabsf(XM) < 1.0e6f)) return;  // non-finite rows: flagged by the logits pass
+  const int T = __float2int_ru(XM) * kLevelsPerOctave;
+  const float deltaf = (float)((double)T / kLevelsPerOctave - (double)XM);  // in [0, 1)
+  // fp32 values of 2^delta and 2^(-1/64) (relative error ~1e-7, inside the slack)
+  const double p_delta = (double)exp2f(deltaf);
+  const double p_64 = (double)exp2f(-1.0f / kLevelsPerOctave);
+  // slack >= 2^E - 1 for E <= 0.5
+  const double slack = (fabs((double)XM) + 2.0 * kMergeOct + 64.0) * 0x1p-22 + 2.5e-5 +
+                       (double)nr * 0x1p-23;
+
+  // coarse merge: octaves O = lane and lane + 32 of the merged frame; range r's
+  // octave o is merged octave O = o - sh_r, sh_r = (top_r - T) / 64.  Ranges go
+  // in rounds of 32: every load of a round is issued before any is used (the
+  // range's octave sums land in registers, octave o in lane o % 32).
+  bool bad = false;
+  float mu[2] = {0.0f, 0.0f};  // fp32 sums of fp32 octave sums (relative error in the slack)
+  double deep = 0.0;  // upper bound of the mass of keys below the merged frame
+  // merges one round of 32 ranges (headers of range r0 + lane in this lane)
+  auto merge_round = [&](int r0, int my_top, uint32_t my_flags, uint32_t my_below,
+                         const float (&oa)[32], const float (&ob)[32]) {
+    const int rl = r0 + lane;
+    const int nb = min(32, nr - r0);
+    bad |= rl < nr && (my_flags != 0u || (my_top % kLevelsPerOctave) != 0);
+    const int my_sh = (rl < nr ? my_top - T : 0) / kLevelsPerOctave;
+    // the range's keys below its own frame: fine index >= kHistBins - 64 sh
+    if (rl < nr && my_below) deep += (double)my_below * p_delta * pow2i(my_sh - kHistOctaves);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j < nb) {
+        const int sh = __shfl_sync(0xffffffffu, my_sh, j);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int o = lane + 32 * k + sh;  // the range octave that merged octave O needs
+          const float va = __shfl_sync(0xffffffffu, oa[j], o & 31);
+          const float vb = __shfl_sync(0xffffffffu, ob[j], o & 31);
+          if (o >= 0 && o < kHistOctaves) mu[k] += (o < 32 ? va : vb);
+        }
+      }
+    }
+    // rare: ranges whose first stage lies so far below the row maximum that
+    // some of their octaves fall below the merged frame (sh <= -17)
+    const uint32_t far = __ballot_sync(0xffffffffu, rl < nr && my_sh <= kHistOctaves - 1 - kMergeOct);
+    for (uint32_t f = far; f; f &= f - 1) {
+      const int j = __ffs(f) - 1;
+      const int sh = __shfl_sync(0xffffffffu, my_sh, j);
+      const RangeHist* h = rh + r0 + j;
+      for (int o = max(kMergeOct + sh, 0) + lane; o < kHistOctaves; o += 32) {
+        const uint32_t c = __ldcg(&h->ocnt[o]);
+        if (c) deep += (double)c * p_delta * pow2i(sh - o);
+      }
+    }
+  };
+  merge_round(0, top0, flags0, below0, oa0, ob0);
+  for (int r0 = 32; r0 < nr; r0 += 32) {  // more than 32 ranges per row (large n)
+    const int rl = r0 + lane;
+    int my_top = 0;
+    uint32_t my_flags = 0u, my_below = 0u;
+    if (rl < nr) {
+      my_top = __ldcg(&rh[rl].top);
+      my_flags = __ldcg(&rh[rl].flags);
+      my_below = __ldcg(&rh[rl].below);
+    }
+    float oa[32], ob[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      oa[j] = 0.0f;
+      ob[j] = 0.0f;
+      if (r0 + j < nr) {
+        oa[j] = __ldcg(&rh[r0 + j].omass[lane]);
+        if (lane + 32 < kHistOctaves) ob[j] = __ldcg(&rh[r0 + j].omass[lane + 32]);
+      }
+    }
+    merge_round(r0, my_top, my_flags, my_below, oa, ob);
+  }
+  if (__any_sync(0xffffffffu, bad)) return;
+  deep = warp_sum_d(deep) * (1.0 + slack);
+  // per-octave mass bounds; octave O holds weights 2^(delta - O - j/64) per unit of omass
+  double hi_m[2], lo_m[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const double f = p_delta * pow2i(-(lane + 32 * k));
+    hi_m[k] = (double)mu[k] * f * (1.0 + slack);
+    lo_m[k] = (double)mu[k] * f * p_64 * (1.0 - slack);
+  }
+  // suffix sums from the bottom of the frame: mass of octaves >= O
+  const double upU = warp_suffix_sum(hi_m[1]), upL = warp_suffix_sum(lo_m[1]);
+  const double totU1 = __shfl_sync(0xffffffffu, upU, 0), totL1 = __shfl_sync(0xffffffffu, upL, 0);
+  const double loU = warp_suffix_sum(hi_m[0]) + totU1, loL = warp_suffix_sum(lo_m[0]) + totL1;
+  const double ZU = __shfl_sync(0xffffffffu, loU, 0) + deep;
+  const double ZL = __shfl_sync(0xffffffffu, loL, 0);
+  const double eps = p.eps;
+  // D+(O) <= eps ZL: the keys of octaves >= O are certainly dropped
+  // D-(O) >  eps ZU: the keys of octaves <  O are certainly kept
+  const double dU[2] = {loU + deep, upU + deep}, dL[2] = {loL, upL};
+  const uint32_t tail0 = __ballot_sync(0xffffffffu, dU[0] <= eps * ZL);
+  const uint32_t tail1 = __ballot_sync(0xffffffffu, dU[1] <= eps * ZL);
+  const uint32_t head0 = __ballot_sync(0xffffffffu, dL[0] > eps * ZU);
+  const uint32_t head1 = __ballot_sync(0xffffffffu, dL[1] > eps * ZU);
+  // smallest O with the tail condition (kMergeOct: only the deep keys;
+  // kMergeOct + 1: none), largest O with the head condition (0 if none)
+  int Olo = tail0 ? __ffs(tail0) - 1 : tail1 ? 32 + __ffs(tail1) - 1
+          : (deep <= eps * ZL ? kMergeOct : kMergeOct + 1);
+  int Ohi = head1 ? 32 + 31 - __clz(head1) : head0 ? 31 - __clz(head0) : 0;
+  if (Olo <= Ohi) return;  // cannot happen with consistent bounds; keep the default
+  // coarse result
+  int g_lo = kLevelsPerOctave * Olo, g_hi = kLevelsPerOctave * Ohi;
+  // fine refinement of the window octaves [Ohi, Olo)
+  const int nwo = Olo - Ohi;
+  if (Olo <= kMergeOct && nwo <= kFineOctMax) {
+    // lane l owns the B = 2 nwo consecutive fine bins g0 + B l ... g0 + B l + B - 1
+    const int B = 2 * nwo;
+    const int g0 = kLevelsPerOctave * Ohi;
+    uint32_t cnt[2 * kFineOctMax];
+#pragma unroll
+    for (int b = 0; b < 2 * kFineOctMax; ++b) cnt[b] = 0u;
+    for (int r0 = 0; r0 < nr; r0 += 32) {
+      const int rl = r0 + lane;
+      const int my_sh =
+          ((rl < nr ? (r0 == 0 ? top0 : __ldcg(&rh[rl].top)) : T) - T) / kLevelsPerOctave;
+      const int nb = min(32, nr - r0);
+#pragma unroll 16
+      for (int j = 0; j < nb; ++j) {
+        const int sh = __shfl_sync(0xffffffffu, my_sh, j);
+        const RangeHist* h = rh + r0 + j;
+        const int gr0 = g0 + B * lane + sh * kLevelsPerOctave;  // the range's fine index
+#pragma unroll
+        for (int b = 0; b < 2 * kFineOctMax; b += 2) {
+          if (b < B) {
+            const int gi = gr0 + b;  // even: one 32-bit load covers bins gi, gi + 1
+            if (gi >= 0 && gi + 1 < kHistBins) {
+              const uint32_t w2 = __ldcg(reinterpret_cast<const unsigned int*>(&h->fine[gi]));
+              cnt[b] += w2 & 0xffffu;
+              cnt[b + 1] += w2 >> 16;
+            }
+          }
+        }
+      }
+    }
+    // per-bin bounds and suffix sums inside the window (bins below it: D(Olo))
+    const double baseU =
+        (Olo < kMergeOct ? __shfl_sync(0xffffffffu, (Olo < 32 ? loU : upU), Olo & 31) : 0.0) + deep;
+    const double baseL =
+        (Olo < kMergeOct) ? __shfl_sync(0xffffffffu, (Olo < 32 ? loL : upL), Olo & 31) : 0.0;
+    double bu[2 * kFineOctMax], bl[2 * kFineOctMax], su = 0.0, sl = 0.0;
+#pragma unroll
+    for (int b = 0; b < 2 * kFineOctMax; ++b) {
+      const int g = g0 + B * lane + b;
+      const double f = p_delta *
+                       (double)exp2f(-(float)(g & (kLevelsPerOctave - 1)) / (float)kLevelsPerOctave) *
+                       pow2i(-(g / kLevelsPerOctave));
+      bu[b] = (b < B) ? (double)cnt[b] * f * (1.0 + slack) : 0.0;
+      bl[b] = (b < B) ? (double)cnt[b] * f * p_64 * (1.0 - slack) : 0.0;
+      su += bu[b];
+      sl += bl[b];
+    }
+    // mass of the window bins of the lanes above this one (larger g)
+    const double aboveU = warp_suffix_sum(su) - su, aboveL = warp_suffix_sum(sl) - sl;
+    // walk this lane's bins from its bottom (largest g) up
+    double DU = baseU + aboveU, DL = baseL + aboveL;
+    int my_lo = INT_MAX, my_hi = -1;
+#pragma unroll
+    for (int b = 2 * kFineOctMax - 1; b >= 0; --b) {
+      if (b < B) {
+        DU += bu[b];
+        DL += bl[b];
+        const int g = g0 + B * lane + b;  // boundary at the top of bin g: keys with index >= g
+        if (DU <= eps * ZL) my_lo = g;
+        if (DL > eps * ZU && my_hi < 0) my_hi = g;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      my_lo = min(my_lo, __shfl_xor_sync(0xffffffffu, my_lo, o));
+      my_hi = max(my_hi, __shfl_xor_sync(0xffffffffu, my_hi, o));
+    }
+    if (my_lo != INT_MAX) g_lo = min(g_lo, my_lo);
+    if (my_hi >= 0) g_hi = max(g_hi, my_hi);
+    if (g_lo <= g_hi) {  // inconsistent: fall back to the coarse window
+      g_lo = kLevelsPerOctave * Olo;
+      g_hi = kLevelsPerOctave * Ohi;
+    }
+  }
+  // keys with fine index >= g_lo (level <= T - g_lo) are dropped, keys with
+  // fine index < g_hi (level > T - g_hi) are kept
+  llo = (Olo > kMergeOct) ? INT_MIN : T - g_lo + 1;
+  lhi = T - g_hi + 1;
+}
+
 template <int RT, bool ERR>
 __global__ void __launch_bounds__(kGThreads, 1)
 gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restrict__ u,
-                 const RowSel* __restrict__ sel, float* __restrict__ acc_out, Plan p,
+                 const float* __restrict__ cmax, TcBufs tb, float* __restrict__ acc_out, Plan p,
                  uint32_t* __restrict__ status) {
-  // the finalisation kernel may be scheduled now; it waits for this grid
+  // the last kernel may be scheduled now; it waits for this grid
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -115,7 +412,9 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
   unsigned char* vring = base;                          // [kGStages][2 boxes][kGK keys][128 B]
   unsigned char* wring = base + kGStages * kGV;         // [kGStages][kGK / 64][kGN rows][128 B]
   float* uring = reinterpret_cast<float*>(wring + kGStages * kGW);  // [kGStages][4 rows][kGK]
-  __shared__ unsigned long long vfull[kGStages], wfull[kGStages], empty[kGStages];
+  unsigned long long* cbuf_all =
+      reinterpret_cast<unsigned long long*>(uring + kGStages * 4 * kGK);  // [4][kCandBuf]
+  __shared__ unsigned long long vfull[kGStages], ufull[kGStages], wfull[kGStages], empty[kGStages];
   __shared__ unsigned long long accfull[2], accempty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
@@ -133,6 +432,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) {
       mbar_init(&vfull[s], 1);
+      mbar_init(&ufull[s], 1);
       mbar_init(&wfull[s], RT);
       mbar_init(&empty[s], 1);
     }
@@ -153,9 +453,22 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       const unsigned long long pol = (p.tiles_out == 1) ? policy_evict_first() : policy_evict_last();
-      const unsigned long long pol_u = policy_evict_first();
+      const unsigned long long pol_u = policy_evict_last();  // read again by the last kernel
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(&vmap))
                    : "memory");
+      // the first ring of value stages goes out before the logits exist
+      int nA = 0;
+      for (int it = blockIdx.x; it < nitems && nA < kGStages; it += gridDim.x) {
+        const GItem g = gitem_of(it, p);
+        const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
+        for (int sg = s_lo; sg < s_hi && nA < kGStages; ++sg, ++nA) {
+          unsigned char* dst = vring + nA * kGV;
+          mbar_arrive_expect_tx(&vfull[nA], (unsigned)kGV);
+          tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[nA], pol);
+          tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[nA], pol);
+        }
+      }
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits pass has completed
       int t = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
@@ -165,33 +478,35 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
         const int nrows = min(RT, p.gm - g.tile * RT);
         for (int sg = s_lo; sg < s_hi; ++sg, ++t) {
           const int slot = t % kGStages;
-          if (t >= kGStages && !mbar_wait(&empty[slot], (unsigned)(t / kGStages - 1) & 1u)) {
-            ok = false;
-            break;
-          }
-          if (aborted(&s_abort)) {
-            ok = false;
-            break;
+          if (t >= nA) {
+            if (!mbar_wait(&empty[slot], (unsigned)(t / kGStages - 1) & 1u) || aborted(&s_abort)) {
+              ok = false;
+              break;
+            }
+            unsigned char* dst = vring + slot * kGV;
+            mbar_arrive_expect_tx(&vfull[slot], (unsigned)kGV);
+            tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[slot], pol);
+            tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[slot], pol);
           }
           // the rows' logits of the stage's keys below n, in whole 16-byte pieces
           // (the logit rows are padded to a multiple of 64 keys)
           const int64_t key0 = (int64_t)sg * kGK;
           const unsigned ub = (unsigned)((min((int64_t)kGK, p.n - key0) + 3) / 4) * 16u;
-          unsigned char* dst = vring + slot * kGV;
-          mbar_arrive_expect_tx(&vfull[slot], (unsigned)kGV + ub * (unsigned)nrows);
-          tma_load_3d(dst, &vmap, 0, (int)key0, g.group, &vfull[slot], pol);
-          tma_load_3d(dst + kGV / 2, &vmap, kGBox, (int)key0, g.group, &vfull[slot], pol);
+          mbar_arrive_expect_tx(&ufull[slot], ub * (unsigned)nrows);
           for (int r = 0; r < nrows; ++r)
             bulk_load(uring + (slot * 4 + r) * kGK, u + (row0 + r) * p.ustride + key0, ub,
-                      &vfull[slot], pol_u);
+                      &ufull[slot], pol_u);
         }
       }
       if (!ok) {
         atomicOr(status, CTA_DEV_TIMEOUT);
         s_abort = 1;
         // the copies still in flight land before the CTA may exit (bounded)
-        for (int t2 = max(0, t - kGStages); t2 < t; ++t2)
+        for (int t2 = max(0, t - kGStages); t2 < t; ++t2) {
           mbar_wait(&vfull[t2 % kGStages], (unsigned)(t2 / kGStages) & 1u);
+          mbar_wait(&ufull[t2 % kGStages], (unsigned)(t2 / kGStages) & 1u);
+        }
+        for (int t2 = t; t2 < nA; ++t2) mbar_wait(&vfull[t2], 0u);
       }
     }
   } else if (warp == 1) {
@@ -240,64 +555,138 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
     // ---------------- weights: warp r -> row r of the tile ----------------
     const int r = warp - kGWeightWarp0;
     if (r < RT) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");  // histograms and maxima are complete
+      const float sc = p.scale2;
       int t = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
         const GItem g = gitem_of(it, p);
         const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
-        const int64_t row0 = (int64_t)g.group * p.gm + (int64_t)g.tile * RT;
+        const int64_t row = (int64_t)g.group * p.gm + (int64_t)g.tile * RT + r;
         const bool row_ok = r < min(RT, p.gm - g.tile * RT);
         float M = 0.0f;
-        uint32_t ks = 0u, is = 0u;
-        // this kernel is a programmatic dependent of selection: its row results
-        // are read only after that grid has finished
-        asm volatile("griddepcontrol.wait;" ::: "memory");
+        int llo = INT_MIN, lhi = INT_MAX;
         if (row_ok) {
-          const RowSel* rs = sel + row0 + r;
-          M = __ldg(&rs->M);
-          ks = __ldg(&rs->kstar);
-          is = (uint32_t)__ldg(&rs->istar);
+          row_bracket(tb.hist, cmax, row, p, M, llo, lhi);
+          if (g.range == 0 && lane == 0) tb.brk[row] = RowBracket{M, llo, lhi, 0u};
         }
+        U128 mz = u128_zero(), mh = u128_zero(), mt = u128_zero();
+        double wh = 0.0, wt = 0.0;  // fp64 sums of per-stage fp32 weight sums (for KL only)
+        uint32_t nh = 0u, nw = 0u;
+        float tmax = kNegInf;
+        unsigned long long* cand = tb.cand + row * kCandCap;
+        unsigned long long* cbuf = cbuf_all + r * kCandBuf;
+        uint32_t nbuf = 0u;
         for (int sg = s_lo; sg < s_hi; ++sg, ++t) {
           const int slot = t % kGStages;
           const int64_t k0 = (int64_t)sg * kGK + 4 * lane;  // this lane's four keys
-          // the stage (values and logits) has landed; its slot's W tile is then
-          // free too (the MMAs that last read the slot have finished)
-          if (!mbar_wait(&vfull[slot], (unsigned)(t / kGStages) & 1u) || aborted(&s_abort)) ok = false;
+          // the stage's logits have landed; its slot's W tile is then free too
+          // (the MMAs that last read the slot have finished)
+          if (!mbar_wait(&ufull[slot], (unsigned)(t / kGStages) & 1u) || aborted(&s_abort)) ok = false;
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
           }
           float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
           if (row_ok) x = reinterpret_cast<const float4*>(uring + (slot * 4 + r) * kGK)[lane];
-          // weights of the four keys, split into kept / dropped and three parts
           uint32_t hp[4][3], tp[4][3];
           const float xs[4] = {x.x, x.y, x.z, x.w};
+          uint32_t winmask = 0u;
+          float sh_ = 0.0f, st_ = 0.0f;
+          // branch-free: every key is kept (level >= lhi), dropped (< llo) or window
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            float w = 0.0f;
-            bool kept = false;
-            if (row_ok && k0 + i < p.n) {
-              w = weight(xs[i], M, p.scale2);
-              kept = is_kept(order_key(xs[i]), (uint32_t)(k0 + i), ks, is);
+            const bool valid = row_ok && k0 + i < p.n;
+            const float w = valid ? weight(xs[i], M, sc) : 0.0f;
+            const int L = key_level(xs[i], sc);
+            const bool head = valid && L >= lhi;
+            const bool tail = valid && L < llo;
+            const unsigned long long W = mass62(w);
+            u128_add(mz, W);
+            u128_add(mh, head ? W : 0ull);
+            u128_add(mt, tail ? W : 0ull);
+            nh += head ? 1u : 0u;
+            nw += (valid && !head && !tail) ? 1u : 0u;
+            winmask |= (valid && !head && !tail) ? (1u << i) : 0u;
+            sh_ += head ? w : 0.0f;
+            st_ += tail ? w : 0.0f;
+            tmax = fmaxf(tmax, tail ? xs[i] : kNegInf);
+            uint32_t pt[3];
+            split3(w, pt);
+#pragma unroll
+            for (int part = 0; part < 3; ++part) {
+              hp[i][part] = head ? pt[part] : 0u;
+              if constexpr (ERR) tp[i][part] = tail ? pt[part] : 0u;
             }
-            split3(kept ? w : 0.0f, hp[i]);
-            if constexpr (ERR) split3(kept ? 0.0f : w, tp[i]);
           }
-          unsigned char* wt = wring + slot * kGW;
+          wh += (double)sh_;
+          wt += (double)st_;
+          unsigned char* wtile = wring + slot * kGW;
           const int c = lane >> 1;  // 16-byte piece (8 keys) along K; this lane writes one half
           const uint32_t half = (uint32_t)(lane & 1) * 8u;
 #pragma unroll
           for (int part = 0; part < 3; ++part) {
-            *reinterpret_cast<uint2*>(wt + sw128_offset(wcol<RT>(0, part, r), c, kGN) + half) =
+            *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(0, part, r), c, kGN) + half) =
                 make_uint2(hp[0][part] | (hp[1][part] << 16), hp[2][part] | (hp[3][part] << 16));
             if constexpr (ERR)
-              *reinterpret_cast<uint2*>(wt + sw128_offset(wcol<RT>(1, part, r), c, kGN) + half) =
+              *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(1, part, r), c, kGN) + half) =
                   make_uint2(tp[0][part] | (tp[1][part] << 16), tp[2][part] | (tp[3][part] << 16));
           }
           fence_proxy_async();
           __syncwarp();
           if (lane == 0) mbar_arrive(&wfull[slot]);
+          // window keys to this warp's buffer (flushed to the row's list when
+          // full and at the end of the item: one global atomic per flush)
+          if (__any_sync(0xffffffffu, winmask != 0u)) {
+            const uint32_t cnt = __popc(winmask);
+            uint32_t pre = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
+              if (lane >= o) pre += y;
+            }
+            const uint32_t total = __shfl_sync(0xffffffffu, pre, 31);
+            if (nbuf + total > (uint32_t)kCandBuf) {
+              flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
+              nbuf = 0u;
+            }
+            uint32_t at = nbuf + pre - cnt;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              if (winmask & (1u << i)) cbuf[at++] = composite(order_key(xs[i]), (uint32_t)(k0 + i));
+            }
+            __syncwarp();
+            nbuf += total;  // a stage adds at most 128 <= kCandBuf keys
+          }
+        }
+        if (row_ok && __any_sync(0xffffffffu, nbuf > 0u)) {
+          flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
+          nbuf = 0u;
+        }
+        if (!ok) break;
+        // the range record of this row
+        mz = u128_warp_sum(mz);
+        mh = u128_warp_sum(mh);
+        mt = u128_warp_sum(mt);
+        const U128 mw = u128_sub(u128_sub(mz, mh), mt);
+        wh = warp_sum_d(wh);
+        wt = warp_sum_d(wt);
+        nh = __reduce_add_sync(0xffffffffu, nh);
+        nw = __reduce_add_sync(0xffffffffu, nw);
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+        if (row_ok && lane == 0) {
+          RangeRec rec;
+          rec.mh = mh;
+          rec.mt = mt;
+          rec.mw = mw;
+          rec.wh = wh;
+          rec.wt = wt;
+          rec.nh = nh;
+          rec.nw = nw;
+          rec.tmax = tmax;
+          rec.pad = 0u;
+          tb.rrec[row * p.nranges + g.range] = rec;
         }
       }
       if (!ok && lane == 0) {
@@ -356,117 +745,35 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
   if (warp == 1) tmem_dealloc(tmem, kGTmemCols);
 }
 
-// Phase 4: one CTA per row, launched as a programmatic dependent of the value
-// pass (it waits for that grid's results).  Thread (a, dim) sums the head
-// (a = 0) or tail (a = 1) partials of one dimension over the ranges in a fixed
-// order, sixteen loads in flight.  256 threads: the CTA fits beside a value-
-// pass or logits CTA on an SM, so it neither waits for a free SM nor keeps the
-// next call's logits pass off one.
-constexpr int kFinThreads = 2 * kGD;
-
-template <bool ERR>
-__global__ void __launch_bounds__(kFinThreads)
-finalize_tc_kernel(const float* __restrict__ acc_out, const RowSel* __restrict__ sel,
-                   const float* __restrict__ gmax, __nv_bfloat16* __restrict__ out,
-                   float* __restrict__ err_out, float* __restrict__ kl_out,
-                   float* __restrict__ gap_out, Plan p, uint32_t* __restrict__ status) {
-  // The next call's logits pass may be scheduled now (it streams K at once
-  // and waits for this grid before it writes the logits).
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ double tail[kGD];
-  __shared__ double sq[kGD];
-  const int64_t row = blockIdx.x;
-  const int tid = threadIdx.x;
-  const int a = tid / kGD, dim = tid % kGD;
-  // every load of the row is issued before the first use: the row's selection
-  // result, its dropped-logit maxima and this thread's range partials
-  const RowSel rs = sel[row];
-  float gpart = kNegInf;  // warp 2 (which forms the gap bound) loads the partial maxima
-  if (tid >= 2 * kWarp && tid - 2 * kWarp < p.gparts)
-    gpart = __ldcg(gmax + row * kMaxGParts + (tid - 2 * kWarp));
-  double s = 0.0;
-  if (ERR || a == 0) {
-    const float* src = acc_out + (row * p.nranges * 2 + a) * kGD + dim;
-#pragma unroll 16
-    for (int c = 0; c < p.nranges; ++c) s += (double)__ldcg(src + (int64_t)c * 2 * kGD);
-  }
-  if (a == 1) tail[dim] = s;
-  __syncthreads();
-  if (a == 0) {
-    const double mu_h = s / rs.wh;
-    out[row * kGD + dim] = __float2bfloat16_rn((float)mu_h);
-    const double diff = (ERR && rs.wt > 0.0) ? tail[dim] / rs.wt - mu_h : 0.0;
-    sq[dim] = diff * diff;
-  }
-  __syncthreads();
-  if (tid < kWarp) {  // fixed-order tree over the dimensions
-    double v = (sq[4 * tid] + sq[4 * tid + 1]) + (sq[4 * tid + 2] + sq[4 * tid + 3]);
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (tid == 0) {
-      if (!(rs.wh > 0.0)) atomicOr(status, CTA_DEV_INTERNAL);
-      if (err_out) err_out[row] = (float)(rs.C < rs.Z && rs.wt > 0.0 ? rs.tv * sqrt(v) : 0.0);
-    }
-  } else if (tid == kWarp) {
-    if (kl_out) kl_out[row] = (float)log1p(rs.wt / rs.wh);
-  } else if (tid >= 2 * kWarp && tid < 3 * kWarp && gap_out) {
-    // the row's largest dropped logit over the selection CTAs' partial maxima
-    float gm = __shfl_sync(0xffffffffu, gpart, 0);
-    for (int c = 1; c < kMaxGParts; ++c) gm = fmaxf(gm, __shfl_sync(0xffffffffu, gpart, c));
-    if (tid == 2 * kWarp)
-      gap_out[row] = (float)single_gap_bound((double)key_value(rs.kstar), (double)gm, rs.k, p.n, kGD);
-  }
-}
-
 template <int RT, bool ERR>
-cudaError_t launch_t(const CUtensorMap& map, const float* u, const RowSel* sel, float* acc,
-                     const Plan& p, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_t(const CUtensorMap& map, const float* u, const float* cmax, const TcBufs& tb,
+                     float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   auto kern = gather_tc_kernel<RT, ERR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
   if (e != cudaSuccess) return e;
   const int sms = sm_count();
   const long long nitems = (long long)p.tiles_out * p.nranges * p.groups;
   const unsigned grid = (unsigned)std::min<long long>(nitems, sms);
-  // programmatic dependent of selection: the value stream starts early
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kGThreads, 1, 1);
   cfg.dynamicSmemBytes = kGSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see "Ordering" above
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, u, sel, acc, p, status);
+  return cudaLaunchKernelEx(&cfg, kern, map, u, cmax, tb, acc, p, status);
 }
 
 template <bool ERR>
-cudaError_t launch_finalize(const float* acc, const RowSel* sel, const float* gmax, void* out,
-                            float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                            uint32_t* status, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.rows, 1, 1);
-  cfg.blockDim = dim3(kFinThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, finalize_tc_kernel<ERR>, acc, sel, gmax,
-                            static_cast<__nv_bfloat16*>(out), err_out, kl_out, gap_out, p, status);
-}
-
-template <bool ERR>
-cudaError_t launch_e(const CUtensorMap& map, const float* u, const RowSel* sel, float* acc,
-                     const Plan& p, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_e(const CUtensorMap& map, const float* u, const float* cmax, const TcBufs& tb,
+                     float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   switch (p.rt_out) {
-    case 1: return launch_t<1, ERR>(map, u, sel, acc, p, status, st);
-    case 2: return launch_t<2, ERR>(map, u, sel, acc, p, status, st);
-    case 4: return launch_t<4, ERR>(map, u, sel, acc, p, status, st);
+    case 1: return launch_t<1, ERR>(map, u, cmax, tb, acc, p, status, st);
+    case 2: return launch_t<2, ERR>(map, u, cmax, tb, acc, p, status, st);
+    case 4: return launch_t<4, ERR>(map, u, cmax, tb, acc, p, status, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -504,8 +811,11 @@ bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The path depends on the shape and dtype alone, so that the workspace size
+// is the same wherever it is computed; a missing tensor-map encoder makes the
+// launch fail (CTA_ERR_CUDA) instead of choosing another path.
 bool gather_tc_applies(const Plan& p, int dtype) {
-  return dtype == kDtypeBF16 && p.d == kGD && p.n >= kGK && p.rt_out <= 4 && encode_tiled() != nullptr;
+  return dtype == kDtypeBF16 && p.d == kGD && p.n >= kGK && p.rt_out <= 4;
 }
 
 void set_ranges_tc(Plan* p, int sms) {
@@ -566,21 +876,13 @@ void set_ranges_tc(Plan* p, int sms) {
   p->nranges = (int)best_nr;
 }
 
-cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
-                             const Plan& p, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_gather_tc(const void* V, const float* u, const float* cmax, const TcBufs& tb,
+                             float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
   if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
-  return p.want_err ? launch_e<true>(map, u, sel, acc, p, status, st)
-                    : launch_e<false>(map, u, sel, acc, p, status, st);
-}
-
-cudaError_t launch_finalize_tc(const float* acc, const RowSel* sel, const float* gmax, void* out,
-                               float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                               uint32_t* status, cudaStream_t st) {
-  return p.want_err
-             ? launch_finalize<true>(acc, sel, gmax, out, err_out, kl_out, gap_out, p, status, st)
-             : launch_finalize<false>(acc, sel, gmax, out, err_out, kl_out, gap_out, p, status, st);
+  return p.want_err ? launch_e<true>(map, u, cmax, tb, acc, p, status, st)
+                    : launch_e<false>(map, u, cmax, tb, acc, p, status, st);
 }
 
 }  // namespace cta

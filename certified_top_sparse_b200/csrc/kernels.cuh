@@ -53,26 +53,29 @@ cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, flo
 // dropped) keys, then (the last CTA of each (KV group, row tile), counted in
 // unit_cnt, which selection zeroes) out, err, KL and the single-gap bound.
 // gather_ctas_per_sm: the CTAs per SM its launch is planned for.
-// Phase 3 on tcgen05 for bf16 values with d = 128 (TMA-fed value stages,
-// weights as the B operand), ranges of 128-key stages chosen by
-// set_ranges_tc(p, SM count); the range partials go to acc as in
-// launch_gather, and launch_finalize_tc forms the outputs.
+// The tensor-core decode path (bf16 q, K, V with d = 128), three kernels:
+//   launch_score_kv_tc: logits (TMA-fed K stages, the row tile's queries as the
+//     B operand), one partial maximum per row and range (Plan::nmax) and the
+//     per-range level histograms; zeroes tb.cand_cnt and tb.ticket;
+//   launch_gather_tc: the value pass after set_ranges_tc: brackets every row's
+//     cut from the histograms, value sums of the keys on either side of the
+//     bracket (range partials in acc), exact masses (tb.rrec), window
+//     candidates (tb.cand) and the brackets (tb.brk);
+//   launch_settle_tc: the exact cut, the kept indices and the outputs.
 bool gather_tc_applies(const Plan& p, int dtype);
-// Phase 1 on tcgen05 for the same problems (bf16 q and K, d = 128), after
-// set_ranges_tc: TMA-fed K stages, the row tile's queries as the B operand;
-// writes the logits and one partial maximum per row and range (Plan::nmax).
-cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cmax, const Plan& p,
-                               uint32_t* status, cudaStream_t st);
+cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cmax,
+                               const TcBufs& tb, const Plan& p, uint32_t* status,
+                               cudaStream_t st);
 // Tensor map of a bf16 [groups][n][128] K or V cache: 128-byte-swizzled boxes
 // of 64 dimensions x 128 keys (the stages of the streaming tensor-core kernels).
 bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p);
 void set_ranges_tc(Plan* p, int sms);
-cudaError_t launch_gather_tc(const void* V, const float* u, const RowSel* sel, float* acc,
-                             const Plan& p, uint32_t* status, cudaStream_t st);
-// Phase 4 after launch_gather_tc: one CTA per row, a programmatic dependent of it.
-cudaError_t launch_finalize_tc(const float* acc, const RowSel* sel, const float* gmax, void* out,
-                               float* err_out, float* kl_out, float* gap_out, const Plan& p,
-                               uint32_t* status, cudaStream_t st);
+cudaError_t launch_gather_tc(const void* V, const float* u, const float* cmax, const TcBufs& tb,
+                             float* acc, const Plan& p, uint32_t* status, cudaStream_t st);
+cudaError_t launch_settle_tc(const void* V, const float* u, const TcBufs& tb, float* acc, void* out,
+                             int32_t* k_out, int32_t* idx_out, float* tv_out, float* err_out,
+                             float* kl_out, float* gap_out, const Plan& p, uint32_t* status,
+                             cudaStream_t st);
 int gather_ctas_per_sm(bool want_err);
 cudaError_t launch_gather(int dtype, const void* V, const float* u, const RowSel* sel, float* acc,
                           uint32_t* unit_cnt, const float* gmax, void* out, float* err_out,

@@ -278,8 +278,13 @@ def test_mass_rounding_cannot_hide_a_large_tail(dtype, d):
     n = 1 << 23
     prob = _sink_over_subquantum_background(n, d, dtype, gap_octaves=40.3)
     g, o, rep = check(prob, 1e-6, f"sink over sub-quantum background {dtype} d={d}")
-    assert o["tv_km1"][0] > 1e-6 and o["k"][0] > 1
-    assert abs(int(g["k"][0]) - int(o["k"][0])) <= 1
+    assert o["tv_km1"][0] > 1e-6 and o["k"][0] > 1 and g["k"][0] > 1
+    # The ~1.35M tied background keys each carry ~7e-13 of the mass; fp32
+    # weights (an exponent of ~40.3 has a unit in the last place of ~4e-6)
+    # move the cut among them by a few keys, which compare() has judged with
+    # the oracle's own masses.  What must not happen is the collapse to k = 1.
+    dropped = prob.n - int(o["k"][0])
+    assert abs(int(g["k"][0]) - int(o["k"][0])) <= 1e-5 * dropped + 1
     assert abs(float(g["tv"][0]) - float(o["tv"][0])) <= 1e-7
 
 
