@@ -226,6 +226,8 @@ struct TcBufs {
   unsigned long long* cand;  // [rows][kCandCap] composite keys of window keys
   uint32_t* cand_cnt;    // [rows] window keys seen (zeroed by the logits pass)
   uint32_t* ticket;      // [rows] ranges settled (zeroed by the logits pass)
+  uint32_t* hmask;       // [rows][mask_words] bit j of word w: key 32 w + j kept for certain
+  int64_t mask_words;    // words per row: 4 per 128-key stage
 };
 
 // ---------------------------------------------------------------------------

@@ -32,7 +32,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct Layout {
   size_t u, cmax, sel, choff, acc, gmax, unit, status;
   // tensor-core decode path only (zero-sized otherwise)
-  size_t hist, rrec, srec, brk, cand, cand_cnt, ticket;
+  size_t hist, rrec, srec, brk, cand, cand_cnt, ticket, hmask;
   size_t total;
 };
 
@@ -103,6 +103,9 @@ int make_plan(int64_t n, int d, int n_heads, int n_kv_heads, int batch, int m, i
   return CTA_OK;
 }
 
+// Words per row of the value pass's kept-key mask: four per 128-key stage.
+int64_t mask_words(const Plan& p) { return 4 * ((p.n + 127) / 128); }
+
 Layout layout(const Plan& p, bool tc_decode) {
   Layout L;
   size_t off = 0;
@@ -123,6 +126,7 @@ Layout layout(const Plan& p, bool tc_decode) {
   L.cand = off;     off = align256(off + sizeof(unsigned long long) * kCandCap * rw);
   L.cand_cnt = off; off = align256(off + sizeof(uint32_t) * rw);
   L.ticket = off;   off = align256(off + sizeof(uint32_t) * rw);
+  L.hmask = off;    off = align256(off + sizeof(uint32_t) * rw * (size_t)mask_words(p));
   L.total = off;
   return L;
 }
@@ -245,6 +249,8 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
     tb.cand = reinterpret_cast<unsigned long long*>(ws + L.cand);
     tb.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cand_cnt);
     tb.ticket = reinterpret_cast<uint32_t*>(ws + L.ticket);
+    tb.hmask = reinterpret_cast<uint32_t*>(ws + L.hmask);
+    tb.mask_words = mask_words(p);
     if (launch_score_kv_tc(q, K, u, cmax, tb, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
     if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
     if (launch_gather_tc(V, u, cmax, tb, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;

@@ -50,8 +50,10 @@
 //              the tensor memory (two accumulators);
 //   warps 2-5  weights: warp r computes row r's bracket once per work item,
 //              then writes row r's part of each stage's W tile and its masses;
-//   warps 6-9  epilogue: read the accumulator, add the parts in fp64, write
-//              the range partial.
+//              at the end of an item the four warps read the accumulator
+//              (each its quarter of the tensor-memory lanes), add the parts in
+//              fp64 and write the range partials.  (Six warps: two per SM
+//              sub-partition at most, so the kernel may use 255 registers.)
 // Work items are (KV group, key range, row tile) with ranges cut in stages so
 // that every SM gets about the same number of stages.
 //
@@ -80,12 +82,11 @@ constexpr int kGBox = 64;             // dimensions per TMA box: 128 bytes of bf
 constexpr int kGV = kGK * kGD * 2;    // value bytes per stage (32 KB)
 constexpr int kGW = kGN * kGK * 2;    // weight-tile bytes per stage (8 KB)
 constexpr int kGU = 4 * kGK * 4;      // logit bytes per stage: up to four rows of kGK fp32 (2 KB)
-constexpr int kGWarps = 10;
+constexpr int kGWarps = 6;
 constexpr int kGThreads = kGWarps * kWarp;
 constexpr int kGWeightWarp0 = 2;
-constexpr int kGEpiWarp0 = 6;
-constexpr int kGEpiThreads = 4 * kWarp;
-constexpr int kGEpiBar = 1;           // named barrier of the epilogue warps
+constexpr int kGEpiThreads = 4 * kWarp;  // the four weight warps also read the accumulator
+constexpr int kGEpiBar = 1;           // named barrier of the weight warps
 constexpr uint32_t kGTmemCols = 2 * kGN;
 constexpr int kCandBuf = 256;         // window keys a weight warp buffers (>= 128: one stage's)
 constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU) + 4 * kCandBuf * 8;
@@ -130,21 +131,6 @@ __device__ __forceinline__ bool aborted(const int* flag) {
   return *reinterpret_cast<const volatile int*>(flag) != 0;
 }
 
-// 2^e exactly, for -1022 <= e <= 1023 (0 below): built from the exponent bits.
-__device__ __forceinline__ double pow2i(int e) {
-  return e < -1022 ? 0.0 : __longlong_as_double((long long)(1023 + min(e, 1023)) << 52);
-}
-
-// Inclusive suffix sums across the lanes (lane l gets the sum over lanes >= l).
-__device__ __forceinline__ double warp_suffix_sum(double v) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double y = __shfl_down_sync(0xffffffffu, v, o);
-    if (lane + o < 32) v += y;
-  }
-  return v;
-}
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -165,44 +151,142 @@ __device__ __forceinline__ void flush_cands(const unsigned long long* buf, uint3
   __syncwarp();
 }
 
+// 2^e in fp32, exactly, for -126 <= e <= 127 (0 below).
+__device__ __forceinline__ float pow2f_int(int e) {
+  return e < -126 ? 0.0f : __int_as_float((127 + min(e, 127)) << 23);
+}
+
+// Inclusive suffix sums across the lanes (lane l gets the sum over lanes >= l).
+__device__ __forceinline__ float warp_suffix_sum_f(float v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_down_sync(0xffffffffu, v, o);
+    v += (lane + o < 32) ? y : 0.0f;
+  }
+  return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Fine counts of the window bins of 32 ranges r0 .. r0 + 31 (ranges >= nr
+// contribute nothing): lane l adds bins g0 + 2 NQ l ... g0 + 2 NQ l + 2 NQ - 1
+// of every range, two per 32-bit load, all loads of the round issued before
+// their sums (no branches: out-of-frame bins are loaded clamped and masked).
+template <int NQ>
+__device__ __forceinline__ void fine_round(const RangeHist* __restrict__ rh, int r0, int nr,
+                                           int my_sh, int g0, uint32_t* cnt) {
+  const int lane = threadIdx.x & 31;
+  constexpr int JC = NQ <= 2 ? 32 : 16;  // ranges per batch of loads (register budget)
+#pragma unroll
+  for (int j0 = 0; j0 < 32; j0 += JC) {
+    uint32_t w[JC][NQ];
+#pragma unroll
+    for (int j = 0; j < JC; ++j) {
+      const int sh = __shfl_sync(0xffffffffu, my_sh, j0 + j);
+      const RangeHist* h = rh + min(r0 + j0 + j, nr - 1);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const int gi = g0 + 2 * NQ * lane + 2 * q + sh * kLevelsPerOctave;  // even
+        const bool ok = r0 + j0 + j < nr && gi >= 0 && gi + 1 < kHistBins;
+        const uint32_t v = __ldcg(reinterpret_cast<const unsigned int*>(
+            &h->fine[min(max(gi, 0), kHistBins - 2)]));
+        w[j][q] = ok ? v : 0u;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < JC; ++j) {
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        cnt[2 * q] += w[j][q] & 0xffffu;
+        cnt[2 * q + 1] += w[j][q] >> 16;
+      }
+    }
+  }
+}
+
+// Merges one round of 32 ranges into the row's merged octave sums mu (octaves
+// lane, lane + 32): range r's octave o is merged octave O = o - sh_r,
+// sh_r = (top_r - T) / 64; the headers of range r0 + lane are in this lane.
+__device__ __forceinline__ void merge_round(const RangeHist* __restrict__ rh, int nr, int T,
+                                            float p_delta, int r0, int my_top, uint32_t my_flags,
+                                            uint32_t my_below, const float (&oa)[32],
+                                            const float (&ob)[32], float (&mu)[2], float& deep,
+                                            bool& bad) {
+  const int lane = threadIdx.x & 31;
+  const bool mine = r0 + lane < nr;
+  bad |= mine && (my_flags != 0u || (my_top % kLevelsPerOctave) != 0);
+  const int my_sh = mine ? (my_top - T) / kLevelsPerOctave : 0;
+  // the range's keys below its own frame: fine index >= kHistBins - 64 sh
+  deep += mine ? (float)my_below * p_delta * pow2f_int(my_sh - kHistOctaves) : 0.0f;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int sh = __shfl_sync(0xffffffffu, my_sh, j);
+    const bool rj = r0 + j < nr;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int o = lane + 32 * k + sh;  // the range octave that merged octave O needs
+      const float va = __shfl_sync(0xffffffffu, oa[j], o & 31);
+      const float vb = __shfl_sync(0xffffffffu, ob[j], o & 31);
+      mu[k] += (rj && o >= 0 && o < kHistOctaves) ? (o < 32 ? va : vb) : 0.0f;
+    }
+  }
+  // rare: ranges whose first stage lies so far below the row maximum that
+  // some of their octaves fall below the merged frame (sh <= -17)
+  const uint32_t far = __ballot_sync(0xffffffffu, mine && my_sh <= kHistOctaves - 1 - kMergeOct);
+  for (uint32_t f = far; f; f &= f - 1) {
+    const int j = __ffs(f) - 1;
+    const int sh = __shfl_sync(0xffffffffu, my_sh, j);
+    const RangeHist* h = rh + r0 + j;
+    for (int o = max(kMergeOct + sh, 0) + lane; o < kHistOctaves; o += 32) {
+      const uint32_t c = __ldcg(&h->ocnt[o]);
+      deep += (float)c * p_delta * pow2f_int(sh - o);
+    }
+  }
+}
+
 // The bracket of one row's cut, computed by one warp from the row's range
 // histograms and range maxima.  Returns (llo, lhi) through the references and
 // the row maximum M.  Every CTA that handles a range of the row computes the
-// same values from the same data.
+// same values from the same data, in the same order.
 //
 // Frame: T = 64 ceil(X_M), X_M = fl(M * scale2), so every key's level is <= T;
 // merged fine index g = T - level, octave O = g / 64.  A key with fine index g
 // has weight w = 2^-a with a within E of X_M - (T - g)/64 ... X_M - (T - g - 1)/64,
 // i.e. 2^(delta - (g + 1)/64) <= w <= 2^(delta - g/64) up to the relative slack
 // s, where delta = T/64 - X_M in [0, 1) and E covers the fp32 rounding of
-// a = (M - u) * scale2 against X_M - x, exp2f's error and the octave sums' own
-// fp32 rounding.
+// a = (M - u) * scale2 against X_M - x and exp2f's error; s also covers the
+// fp32 arithmetic of the bounds themselves (sums of at most ~3000 terms).
+// Every loop is branch-free and fully unrolled so that its loads and
+// shuffles overlap.
 __device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __restrict__ cmax,
-                            int64_t row, const Plan& p, float& M_out, int& llo, int& lhi) {
+                            int64_t row, const Plan& p, float& M_out, int& llo, int& lhi,
+                            unsigned long long* loads_done) {
   const int lane = threadIdx.x & 31;
   const int nr = p.nranges;
   const RangeHist* rh = hist + row * nr;
+  // lane 0 signals (once) when the bracket's loads no longer wait behind the value stream
+  bool signalled = loads_done == nullptr;
+  auto signal = [&]() {
+    if (!signalled && lane == 0) mbar_arrive(loads_done);
+    signalled = true;
+  };
   // Round 0 of the loads, all issued before any is used: the range maxima, the
   // headers and the octave sums of ranges 0 .. 31 (octave o in lane o % 32).
-  int top0 = 0;
-  uint32_t flags0 = 0u, below0 = 0u;
+  const int rl0 = min(lane, nr - 1);
+  float M = __ldcg(cmax + row * p.nchunks + rl0);
+  const int top0 = __ldcg(&rh[rl0].top);
+  const uint32_t flags0 = __ldcg(&rh[rl0].flags);
+  const uint32_t below0 = __ldcg(&rh[rl0].below);
   float oa0[32], ob0[32];
-  const int nb0 = min(32, nr);
-  float M = kNegInf;
-  if (lane < nr) {
-    M = __ldcg(cmax + row * p.nchunks + lane);
-    top0 = __ldcg(&rh[lane].top);
-    flags0 = __ldcg(&rh[lane].flags);
-    below0 = __ldcg(&rh[lane].below);
-  }
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
-    oa0[j] = 0.0f;
-    ob0[j] = 0.0f;
-    if (j < nb0) {
-      oa0[j] = __ldcg(&rh[j].omass[lane]);
-      if (lane + 32 < kHistOctaves) ob0[j] = __ldcg(&rh[j].omass[lane + 32]);
-    }
+    const RangeHist* h = rh + min(j, nr - 1);
+    oa0[j] = __ldcg(&h->omass[lane]);
+    ob0[j] = __ldcg(&h->omass[min(lane + 32, kHistOctaves - 1)]);
   }
   for (int r = 32 + lane; r < nr; r += 32) M = fmaxf(M, __ldcg(cmax + row * p.nchunks + r));
 #pragma unroll
@@ -211,112 +295,70 @@ __device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __r
   llo = INT_MIN;  // defaults: every key is in the window
   lhi = INT_MAX;
   const float XM = __fmul_rn(M, p.scale2);
-  if (!(fabsf(XM) < 1.0e6f)) return;  // non-finite rows: flagged by the logits pass
+  if (!(fabsf(XM) < 1.0e6f)) {  // non-finite rows: flagged by the logits pass
+    signal();
+    return;
+  }
   const int T = __float2int_ru(XM) * kLevelsPerOctave;
-  const float deltaf = (float)((double)T / kLevelsPerOctave - (double)XM);  // in [0, 1)
-  // fp32 values of 2^delta and 2^(-1/64) (relative error ~1e-7, inside the slack)
-  const double p_delta = (double)exp2f(deltaf);
-  const double p_64 = (double)exp2f(-1.0f / kLevelsPerOctave);
-  // slack >= 2^E - 1 for E <= 0.5
-  const double slack = (fabs((double)XM) + 2.0 * kMergeOct + 64.0) * 0x1p-22 + 2.5e-5 +
-                       (double)nr * 0x1p-23;
+  const float delta = (float)((double)T / kLevelsPerOctave - (double)XM);  // in [0, 1)
+  const float p_delta = exp2f(delta);
+  const float p_64 = exp2f(-1.0f / kLevelsPerOctave);
+  const float slack = (fabsf(XM) + 2.0f * kMergeOct + 64.0f) * 0x1p-22f + 1.0e-4f;
 
-  // coarse merge: octaves O = lane and lane + 32 of the merged frame; range r's
-  // octave o is merged octave O = o - sh_r, sh_r = (top_r - T) / 64.  Ranges go
-  // in rounds of 32: every load of a round is issued before any is used (the
-  // range's octave sums land in registers, octave o in lane o % 32).
+  // coarse merge: octaves O = lane and lane + 32 of the merged frame
   bool bad = false;
-  float mu[2] = {0.0f, 0.0f};  // fp32 sums of fp32 octave sums (relative error in the slack)
-  double deep = 0.0;  // upper bound of the mass of keys below the merged frame
-  // merges one round of 32 ranges (headers of range r0 + lane in this lane)
-  auto merge_round = [&](int r0, int my_top, uint32_t my_flags, uint32_t my_below,
-                         const float (&oa)[32], const float (&ob)[32]) {
-    const int rl = r0 + lane;
-    const int nb = min(32, nr - r0);
-    bad |= rl < nr && (my_flags != 0u || (my_top % kLevelsPerOctave) != 0);
-    const int my_sh = (rl < nr ? my_top - T : 0) / kLevelsPerOctave;
-    // the range's keys below its own frame: fine index >= kHistBins - 64 sh
-    if (rl < nr && my_below) deep += (double)my_below * p_delta * pow2i(my_sh - kHistOctaves);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < nb) {
-        const int sh = __shfl_sync(0xffffffffu, my_sh, j);
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int o = lane + 32 * k + sh;  // the range octave that merged octave O needs
-          const float va = __shfl_sync(0xffffffffu, oa[j], o & 31);
-          const float vb = __shfl_sync(0xffffffffu, ob[j], o & 31);
-          if (o >= 0 && o < kHistOctaves) mu[k] += (o < 32 ? va : vb);
-        }
-      }
-    }
-    // rare: ranges whose first stage lies so far below the row maximum that
-    // some of their octaves fall below the merged frame (sh <= -17)
-    const uint32_t far = __ballot_sync(0xffffffffu, rl < nr && my_sh <= kHistOctaves - 1 - kMergeOct);
-    for (uint32_t f = far; f; f &= f - 1) {
-      const int j = __ffs(f) - 1;
-      const int sh = __shfl_sync(0xffffffffu, my_sh, j);
-      const RangeHist* h = rh + r0 + j;
-      for (int o = max(kMergeOct + sh, 0) + lane; o < kHistOctaves; o += 32) {
-        const uint32_t c = __ldcg(&h->ocnt[o]);
-        if (c) deep += (double)c * p_delta * pow2i(sh - o);
-      }
-    }
-  };
-  merge_round(0, top0, flags0, below0, oa0, ob0);
+  float mu[2] = {0.0f, 0.0f};
+  float deep = 0.0f;  // upper bound of the mass of keys below the merged frame
+  merge_round(rh, nr, T, p_delta, 0, top0, flags0, below0, oa0, ob0, mu, deep, bad);
   for (int r0 = 32; r0 < nr; r0 += 32) {  // more than 32 ranges per row (large n)
-    const int rl = r0 + lane;
-    int my_top = 0;
-    uint32_t my_flags = 0u, my_below = 0u;
-    if (rl < nr) {
-      my_top = __ldcg(&rh[rl].top);
-      my_flags = __ldcg(&rh[rl].flags);
-      my_below = __ldcg(&rh[rl].below);
-    }
+    const int rl = min(r0 + lane, nr - 1);
+    const int my_top = __ldcg(&rh[rl].top);
+    const uint32_t my_flags = __ldcg(&rh[rl].flags), my_below = __ldcg(&rh[rl].below);
     float oa[32], ob[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      oa[j] = 0.0f;
-      ob[j] = 0.0f;
-      if (r0 + j < nr) {
-        oa[j] = __ldcg(&rh[r0 + j].omass[lane]);
-        if (lane + 32 < kHistOctaves) ob[j] = __ldcg(&rh[r0 + j].omass[lane + 32]);
-      }
+      const RangeHist* h = rh + min(r0 + j, nr - 1);
+      oa[j] = __ldcg(&h->omass[lane]);
+      ob[j] = __ldcg(&h->omass[min(lane + 32, kHistOctaves - 1)]);
     }
-    merge_round(r0, my_top, my_flags, my_below, oa, ob);
+    merge_round(rh, nr, T, p_delta, r0, my_top, my_flags, my_below, oa, ob, mu, deep, bad);
   }
-  if (__any_sync(0xffffffffu, bad)) return;
-  deep = warp_sum_d(deep) * (1.0 + slack);
+  if (__any_sync(0xffffffffu, bad)) {
+    signal();
+    return;
+  }
+  deep = warp_sum_f(deep) * (1.0f + slack);
   // per-octave mass bounds; octave O holds weights 2^(delta - O - j/64) per unit of omass
-  double hi_m[2], lo_m[2];
+  float hi_m[2], lo_m[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
-    const double f = p_delta * pow2i(-(lane + 32 * k));
-    hi_m[k] = (double)mu[k] * f * (1.0 + slack);
-    lo_m[k] = (double)mu[k] * f * p_64 * (1.0 - slack);
+    const float f = p_delta * pow2f_int(-(lane + 32 * k));
+    hi_m[k] = mu[k] * f * (1.0f + slack);
+    lo_m[k] = mu[k] * f * p_64 * (1.0f - slack);
   }
   // suffix sums from the bottom of the frame: mass of octaves >= O
-  const double upU = warp_suffix_sum(hi_m[1]), upL = warp_suffix_sum(lo_m[1]);
-  const double totU1 = __shfl_sync(0xffffffffu, upU, 0), totL1 = __shfl_sync(0xffffffffu, upL, 0);
-  const double loU = warp_suffix_sum(hi_m[0]) + totU1, loL = warp_suffix_sum(lo_m[0]) + totL1;
-  const double ZU = __shfl_sync(0xffffffffu, loU, 0) + deep;
-  const double ZL = __shfl_sync(0xffffffffu, loL, 0);
-  const double eps = p.eps;
+  const float upU = warp_suffix_sum_f(hi_m[1]), upL = warp_suffix_sum_f(lo_m[1]);
+  const float totU1 = __shfl_sync(0xffffffffu, upU, 0), totL1 = __shfl_sync(0xffffffffu, upL, 0);
+  const float loU = warp_suffix_sum_f(hi_m[0]) + totU1, loL = warp_suffix_sum_f(lo_m[0]) + totL1;
+  const float ZU = __shfl_sync(0xffffffffu, loU, 0) + deep;
+  const float ZL = __shfl_sync(0xffffffffu, loL, 0);
+  const float eps = (float)p.eps;
   // D+(O) <= eps ZL: the keys of octaves >= O are certainly dropped
   // D-(O) >  eps ZU: the keys of octaves <  O are certainly kept
-  const double dU[2] = {loU + deep, upU + deep}, dL[2] = {loL, upL};
-  const uint32_t tail0 = __ballot_sync(0xffffffffu, dU[0] <= eps * ZL);
-  const uint32_t tail1 = __ballot_sync(0xffffffffu, dU[1] <= eps * ZL);
-  const uint32_t head0 = __ballot_sync(0xffffffffu, dL[0] > eps * ZU);
-  const uint32_t head1 = __ballot_sync(0xffffffffu, dL[1] > eps * ZU);
+  const uint32_t tail0 = __ballot_sync(0xffffffffu, loU + deep <= eps * ZL);
+  const uint32_t tail1 = __ballot_sync(0xffffffffu, upU + deep <= eps * ZL);
+  const uint32_t head0 = __ballot_sync(0xffffffffu, loL > eps * ZU);
+  const uint32_t head1 = __ballot_sync(0xffffffffu, upL > eps * ZU);
   // smallest O with the tail condition (kMergeOct: only the deep keys;
   // kMergeOct + 1: none), largest O with the head condition (0 if none)
-  int Olo = tail0 ? __ffs(tail0) - 1 : tail1 ? 32 + __ffs(tail1) - 1
-          : (deep <= eps * ZL ? kMergeOct : kMergeOct + 1);
-  int Ohi = head1 ? 32 + 31 - __clz(head1) : head0 ? 31 - __clz(head0) : 0;
-  if (Olo <= Ohi) return;  // cannot happen with consistent bounds; keep the default
-  // coarse result
-  int g_lo = kLevelsPerOctave * Olo, g_hi = kLevelsPerOctave * Ohi;
+  const int Olo = tail0 ? __ffs(tail0) - 1 : tail1 ? 32 + __ffs(tail1) - 1
+                : (deep <= eps * ZL ? kMergeOct : kMergeOct + 1);
+  const int Ohi = head1 ? 32 + 31 - __clz(head1) : head0 ? 31 - __clz(head0) : 0;
+  if (Olo <= Ohi) {  // cannot happen with consistent bounds; keep the default
+    signal();
+    return;
+  }
+  int g_lo = kLevelsPerOctave * Olo, g_hi = kLevelsPerOctave * Ohi;  // the coarse result
   // fine refinement of the window octaves [Ohi, Olo)
   const int nwo = Olo - Ohi;
   if (Olo <= kMergeOct && nwo <= kFineOctMax) {
@@ -327,59 +369,46 @@ __device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __r
 #pragma unroll
     for (int b = 0; b < 2 * kFineOctMax; ++b) cnt[b] = 0u;
     for (int r0 = 0; r0 < nr; r0 += 32) {
-      const int rl = r0 + lane;
       const int my_sh =
-          ((rl < nr ? (r0 == 0 ? top0 : __ldcg(&rh[rl].top)) : T) - T) / kLevelsPerOctave;
-      const int nb = min(32, nr - r0);
-#pragma unroll 16
-      for (int j = 0; j < nb; ++j) {
-        const int sh = __shfl_sync(0xffffffffu, my_sh, j);
-        const RangeHist* h = rh + r0 + j;
-        const int gr0 = g0 + B * lane + sh * kLevelsPerOctave;  // the range's fine index
-#pragma unroll
-        for (int b = 0; b < 2 * kFineOctMax; b += 2) {
-          if (b < B) {
-            const int gi = gr0 + b;  // even: one 32-bit load covers bins gi, gi + 1
-            if (gi >= 0 && gi + 1 < kHistBins) {
-              const uint32_t w2 = __ldcg(reinterpret_cast<const unsigned int*>(&h->fine[gi]));
-              cnt[b] += w2 & 0xffffu;
-              cnt[b + 1] += w2 >> 16;
-            }
-          }
-        }
+          ((r0 == 0 ? top0 : __ldcg(&rh[min(r0 + lane, nr - 1)].top)) - T) / kLevelsPerOctave;
+      switch (nwo) {
+        case 1: fine_round<1>(rh, r0, nr, my_sh, g0, cnt); break;
+        case 2: fine_round<2>(rh, r0, nr, my_sh, g0, cnt); break;
+        case 3: fine_round<3>(rh, r0, nr, my_sh, g0, cnt); break;
+        default: fine_round<4>(rh, r0, nr, my_sh, g0, cnt); break;
       }
     }
+    signal();
     // per-bin bounds and suffix sums inside the window (bins below it: D(Olo))
-    const double baseU =
-        (Olo < kMergeOct ? __shfl_sync(0xffffffffu, (Olo < 32 ? loU : upU), Olo & 31) : 0.0) + deep;
-    const double baseL =
-        (Olo < kMergeOct) ? __shfl_sync(0xffffffffu, (Olo < 32 ? loL : upL), Olo & 31) : 0.0;
-    double bu[2 * kFineOctMax], bl[2 * kFineOctMax], su = 0.0, sl = 0.0;
+    const float baseU =
+        (Olo < kMergeOct ? __shfl_sync(0xffffffffu, (Olo < 32 ? loU : upU), Olo & 31) : 0.0f) + deep;
+    const float baseL =
+        (Olo < kMergeOct) ? __shfl_sync(0xffffffffu, (Olo < 32 ? loL : upL), Olo & 31) : 0.0f;
+    float bu[2 * kFineOctMax], bl[2 * kFineOctMax], su = 0.0f, sl = 0.0f;
 #pragma unroll
     for (int b = 0; b < 2 * kFineOctMax; ++b) {
       const int g = g0 + B * lane + b;
-      const double f = p_delta *
-                       (double)exp2f(-(float)(g & (kLevelsPerOctave - 1)) / (float)kLevelsPerOctave) *
-                       pow2i(-(g / kLevelsPerOctave));
-      bu[b] = (b < B) ? (double)cnt[b] * f * (1.0 + slack) : 0.0;
-      bl[b] = (b < B) ? (double)cnt[b] * f * p_64 * (1.0 - slack) : 0.0;
+      const float f = p_delta *
+                      exp2f(-(float)(g & (kLevelsPerOctave - 1)) / (float)kLevelsPerOctave) *
+                      pow2f_int(-(g / kLevelsPerOctave));
+      bu[b] = (b < B) ? (float)cnt[b] * f * (1.0f + slack) : 0.0f;
+      bl[b] = (b < B) ? (float)cnt[b] * f * p_64 * (1.0f - slack) : 0.0f;
       su += bu[b];
       sl += bl[b];
     }
     // mass of the window bins of the lanes above this one (larger g)
-    const double aboveU = warp_suffix_sum(su) - su, aboveL = warp_suffix_sum(sl) - sl;
+    const float aboveU = warp_suffix_sum_f(su) - su, aboveL = warp_suffix_sum_f(sl) - sl;
     // walk this lane's bins from its bottom (largest g) up
-    double DU = baseU + aboveU, DL = baseL + aboveL;
+    float DU = baseU + aboveU, DL = baseL + aboveL;
     int my_lo = INT_MAX, my_hi = -1;
 #pragma unroll
     for (int b = 2 * kFineOctMax - 1; b >= 0; --b) {
-      if (b < B) {
-        DU += bu[b];
-        DL += bl[b];
-        const int g = g0 + B * lane + b;  // boundary at the top of bin g: keys with index >= g
-        if (DU <= eps * ZL) my_lo = g;
-        if (DL > eps * ZU && my_hi < 0) my_hi = g;
-      }
+      DU += bu[b];
+      DL += bl[b];
+      const int g = g0 + B * lane + b;  // boundary at the top of bin g: keys with index >= g
+      const bool in = b < B;
+      my_lo = (in && DU <= eps * ZL) ? g : my_lo;
+      my_hi = (in && DL > eps * ZU && my_hi < 0) ? g : my_hi;
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) {
@@ -393,6 +422,7 @@ __device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __r
       g_hi = kLevelsPerOctave * Ohi;
     }
   }
+  signal();
   // keys with fine index >= g_lo (level <= T - g_lo) are dropped, keys with
   // fine index < g_hi (level > T - g_hi) are kept
   llo = (Olo > kMergeOct) ? INT_MIN : T - g_lo + 1;
@@ -416,6 +446,8 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       reinterpret_cast<unsigned long long*>(uring + kGStages * 4 * kGK);  // [4][kCandBuf]
   __shared__ unsigned long long vfull[kGStages], ufull[kGStages], wfull[kGStages], empty[kGStages];
   __shared__ unsigned long long accfull[2], accempty[2], drain;
+  // the first item's bracket loads have returned: the value stream may start
+  __shared__ unsigned long long brk_loads;
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
 
@@ -441,6 +473,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       mbar_init(&accempty[b], kGEpiThreads);
     }
     mbar_init(&drain, 1);
+    mbar_init(&brk_loads, 4);  // one arrival per weight warp
     s_abort = 0;
     mbar_fence_init();
   }
@@ -456,7 +489,10 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       const unsigned long long pol_u = policy_evict_last();  // read again by the last kernel
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(&vmap))
                    : "memory");
-      // the first ring of value stages goes out before the logits exist
+      // The first ring of value stages goes out before the logits exist, once
+      // the weight warps' bracket loads are back: the flood of value loads
+      // would otherwise stretch their latency (bounded wait, then go anyway).
+      mbar_wait(&brk_loads, 0u);
       int nA = 0;
       for (int it = blockIdx.x; it < nitems && nA < kGStages; it += gridDim.x) {
         const GItem g = gitem_of(it, p);
@@ -551,23 +587,32 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       tc_commit(&drain);  // every MMA issued has finished before the CTA exits (bounded)
       mbar_wait(&drain, 0u);
     }
-  } else if (warp < kGEpiWarp0) {
-    // ---------------- weights: warp r -> row r of the tile ----------------
+  } else {
+    // ---------------- weights: warp r -> row r of the tile; accumulator ----------------
     const int r = warp - kGWeightWarp0;
-    if (r < RT) {
+    // warps without a row in the first item let the value stream start at once
+    const bool first_row = r < RT && blockIdx.x < nitems &&
+                           r < min(RT, p.gm - gitem_of(blockIdx.x, p).tile * RT);
+    if (!first_row && lane == 0) mbar_arrive(&brk_loads);
+    const int quarter = warp & 3;  // TMEM lanes (dimensions) this warp may read
+    const int dim = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+    {
       asm volatile("griddepcontrol.wait;" ::: "memory");  // histograms and maxima are complete
       const float sc = p.scale2;
-      int t = 0;
+      int t = 0, jj = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++jj) {
         const GItem g = gitem_of(it, p);
         const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
         const int64_t row = (int64_t)g.group * p.gm + (int64_t)g.tile * RT + r;
-        const bool row_ok = r < min(RT, p.gm - g.tile * RT);
+        const int nrows = min(RT, p.gm - g.tile * RT);
+        const bool row_ok = r < nrows;
         float M = 0.0f;
         int llo = INT_MIN, lhi = INT_MAX;
         if (row_ok) {
-          row_bracket(tb.hist, cmax, row, p, M, llo, lhi);
+          row_bracket(tb.hist, cmax, row, p, M, llo, lhi,
+                      it == (int)blockIdx.x ? &brk_loads : nullptr);
           if (g.range == 0 && lane == 0) tb.brk[row] = RowBracket{M, llo, lhi, 0u};
         }
         U128 mz = u128_zero(), mh = u128_zero(), mt = u128_zero();
@@ -577,7 +622,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
         unsigned long long* cand = tb.cand + row * kCandCap;
         unsigned long long* cbuf = cbuf_all + r * kCandBuf;
         uint32_t nbuf = 0u;
-        for (int sg = s_lo; sg < s_hi; ++sg, ++t) {
+        for (int sg = s_lo; sg < s_hi && r < RT && ok; ++sg, ++t) {
           const int slot = t % kGStages;
           const int64_t k0 = (int64_t)sg * kGK + 4 * lane;  // this lane's four keys
           // the stage's logits have landed; its slot's W tile is then free too
@@ -591,7 +636,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
           if (row_ok) x = reinterpret_cast<const float4*>(uring + (slot * 4 + r) * kGK)[lane];
           uint32_t hp[4][3], tp[4][3];
           const float xs[4] = {x.x, x.y, x.z, x.w};
-          uint32_t winmask = 0u;
+          uint32_t winmask = 0u, hbits = 0u;
           float sh_ = 0.0f, st_ = 0.0f;
           // branch-free: every key is kept (level >= lhi), dropped (< llo) or window
 #pragma unroll
@@ -606,6 +651,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
             u128_add(mh, head ? W : 0ull);
             u128_add(mt, tail ? W : 0ull);
             nh += head ? 1u : 0u;
+            hbits |= head ? (1u << i) : 0u;
             nw += (valid && !head && !tail) ? 1u : 0u;
             winmask |= (valid && !head && !tail) ? (1u << i) : 0u;
             sh_ += head ? w : 0.0f;
@@ -621,6 +667,15 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
           }
           wh += (double)sh_;
           wt += (double)st_;
+          // the stage's kept-for-certain bits: lane l holds keys 4 l .. 4 l + 3,
+          // i.e. bits 4 (l % 8) .. of word l / 8; eight lanes OR their nibbles
+          {
+            uint32_t wv = hbits << (4 * (lane & 7));
+            wv |= __shfl_xor_sync(0xffffffffu, wv, 1);
+            wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
+            wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
+            if (row_ok && (lane & 7) == 0) tb.hmask[row * tb.mask_words + 4 * (int64_t)sg + (lane >> 3)] = wv;
+          }
           unsigned char* wtile = wring + slot * kGW;
           const int c = lane >> 1;  // 16-byte piece (8 keys) along K; this lane writes one half
           const uint32_t half = (uint32_t)(lane & 1) * 8u;
@@ -663,78 +718,64 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
           flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
           nbuf = 0u;
         }
-        if (!ok) break;
-        // the range record of this row
-        mz = u128_warp_sum(mz);
-        mh = u128_warp_sum(mh);
-        mt = u128_warp_sum(mt);
-        const U128 mw = u128_sub(u128_sub(mz, mh), mt);
-        wh = warp_sum_d(wh);
-        wt = warp_sum_d(wt);
-        nh = __reduce_add_sync(0xffffffffu, nh);
-        nw = __reduce_add_sync(0xffffffffu, nw);
+        if (ok) {
+          // the range record of this row
+          mz = u128_warp_sum(mz);
+          mh = u128_warp_sum(mh);
+          mt = u128_warp_sum(mt);
+          const U128 mw = u128_sub(u128_sub(mz, mh), mt);
+          wh = warp_sum_d(wh);
+          wt = warp_sum_d(wt);
+          nh = __reduce_add_sync(0xffffffffu, nh);
+          nw = __reduce_add_sync(0xffffffffu, nw);
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-        if (row_ok && lane == 0) {
-          RangeRec rec;
-          rec.mh = mh;
-          rec.mt = mt;
-          rec.mw = mw;
-          rec.wh = wh;
-          rec.wt = wt;
-          rec.nh = nh;
-          rec.nw = nw;
-          rec.tmax = tmax;
-          rec.pad = 0u;
-          tb.rrec[row * p.nranges + g.range] = rec;
+          for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+          if (row_ok && lane == 0) {
+            RangeRec rec;
+            rec.mh = mh;
+            rec.mt = mt;
+            rec.mw = mw;
+            rec.wh = wh;
+            rec.wt = wt;
+            rec.nh = nh;
+            rec.nw = nw;
+            rec.tmax = tmax;
+            rec.pad = 0u;
+            tb.rrec[row * p.nranges + g.range] = rec;
+          }
+        }
+        // the accumulator of the item: each warp its 32 dimensions of every row,
+        // the three parts added in fp64, fixed order
+        const int b = jj & 1;
+        const bool acc_ok = ok && mbar_wait(&accfull[b], (unsigned)(jj >> 1) & 1u) && !aborted(&s_abort);
+        if (bar_red_or(kGEpiBar, kGEpiThreads, !acc_ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        __syncwarp();
+        uint32_t c[32];
+        tc_ld32(lane_addr + (uint32_t)(b * kGN), c);
+        tc_fence_before();
+        mbar_arrive(&accempty[b]);
+        const int64_t row0 = (int64_t)g.group * p.gm + (int64_t)g.tile * RT;
+#pragma unroll
+        for (int rr = 0; rr < RT; ++rr) {
+          if (rr < nrows) {
+#pragma unroll
+            for (int a = 0; a < (ERR ? 2 : 1); ++a) {
+              const double v = ((double)__uint_as_float(c[wcol<RT>(a, 0, rr)]) +
+                                (double)__uint_as_float(c[wcol<RT>(a, 1, rr)])) +
+                               (double)__uint_as_float(c[wcol<RT>(a, 2, rr)]);
+              acc_out[(((row0 + rr) * p.nranges + g.range) * 2 + a) * kGD + dim] = (float)v;
+            }
+          }
         }
       }
       if (!ok && lane == 0) {
         atomicOr(status, CTA_DEV_TIMEOUT);
         s_abort = 1;
       }
-    }
-  } else {
-    // ---------------- epilogue ----------------
-    const int tid = threadIdx.x - kGEpiWarp0 * kWarp;  // 0..127
-    const int quarter = warp & 3;                      // TMEM lanes this warp may read
-    const int dim = quarter * 32 + lane;
-    const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    int j = 0;
-    bool failed = false;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++j) {
-      const GItem g = gitem_of(it, p);
-      const int64_t row0 = (int64_t)g.group * p.gm + (int64_t)g.tile * RT;
-      const int nrows = min(RT, p.gm - g.tile * RT);
-      const int b = j & 1;
-      const bool ok = mbar_wait(&accfull[b], (unsigned)(j >> 1) & 1u);
-      if (bar_red_or(kGEpiBar, kGEpiThreads, !ok || aborted(&s_abort))) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
-      __syncwarp();
-      uint32_t c[32];
-      tc_ld32(lane_addr + (uint32_t)(b * kGN), c);
-      tc_fence_before();
-      mbar_arrive(&accempty[b]);
-      // range partial of each row: the three parts added in fp64, fixed order
-#pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        if (r < nrows) {
-#pragma unroll
-          for (int a = 0; a < (ERR ? 2 : 1); ++a) {
-            const double v = ((double)__uint_as_float(c[wcol<RT>(a, 0, r)]) +
-                              (double)__uint_as_float(c[wcol<RT>(a, 1, r)])) +
-                             (double)__uint_as_float(c[wcol<RT>(a, 2, r)]);
-            acc_out[(((row0 + r) * p.nranges + g.range) * 2 + a) * kGD + dim] = (float)v;
-          }
-        }
-      }
-    }
-    if (failed && tid == 0) {
-      atomicOr(status, CTA_DEV_TIMEOUT);
-      s_abort = 1;
     }
   }
 
@@ -823,7 +864,9 @@ void set_ranges_tc(Plan* p, int sms) {
   const int64_t spu = (p->n + kGK - 1) / kGK;
   // range partials fit the workspace (one slot per chunk); at most 1024 ranges are tried
   const int64_t cap = std::min<int64_t>(std::min<int64_t>(spu, p->nchunks), 1024);
-  constexpr int64_t kItemCost = 1;  // a stage's worth of hand-over per item
+  // A work item starts with the row bracket (a few microseconds: about ten
+  // stages of streaming), so the planner charges that much per item.
+  constexpr int64_t kItemCost = 10;
   // Every range count is scored by the busiest CTA's items times their length
   // (items go round-robin over the grid); the eight best are then simulated
   // exactly (the last range of a unit is shorter).

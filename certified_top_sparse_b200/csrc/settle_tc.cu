@@ -61,6 +61,8 @@ constexpr int kMaxGroup = 32;            // value-pass ranges per CTA
 constexpr int kSubMax = 512;             // sub-level bins of the cut search
 constexpr int kSubList = 256;            // keys of the cut's sub-level that are sorted
 constexpr int kWList = 256;              // per-warp list of window keys awaiting their value rows
+constexpr int kMaskBlock = 4 * kTThreads;  // mask words per block of the index writes (4 per thread)
+constexpr int kVPre = 64;                // window value rows copied in while the cut is searched
 
 struct SettleShared {
   unsigned long long cand[kCandCap];     // the row's candidates (sorted in place by the fallback)
@@ -75,7 +77,14 @@ struct SettleShared {
       unsigned long long lo[256], hi[256];  // radix digit masses, 128-bit
       uint32_t cnt[256];
     } rx;
+    struct {
+      uint32_t win[kMaskBlock];   // kept window keys of a block of mask words
+      uint32_t word[kMaskBlock];  // kept keys of the block
+      uint32_t off[kMaskBlock];   // exclusive offsets of the words' kept keys
+    } mk;
   } u;
+  uint32_t mask0[kMaskBlock];            // the segment's first block of kept-for-certain words
+  uint2 vrow[kVPre][kTD / 4];            // value rows of the segment's first window keys
   unsigned long long wl_key[kTWarps][kWList];  // window key: logit bits (high 32) | index (low 32)
   unsigned char wl_kept[kTWarps][kWList];
   float accw[2][kTWarps][kTD];           // per-warp window value sums (kept, dropped)
@@ -88,9 +97,22 @@ struct SettleShared {
   uint32_t NH, NHbefore, NW, ccnt, cabove, nsl, off_win;
   unsigned long long cut;
   long long k;
-  uint32_t okmin, okmax;                 // order keys of the lowest and highest candidate
+  uint32_t nlist;
   int found, jstar, last;
 };
+
+// 16-byte asynchronous copy global -> shared (L2 only), and its group waits.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 __device__ __forceinline__ U128 u128_make(unsigned long long lo, unsigned long long hi) {
   return U128{lo, hi};
@@ -232,14 +254,19 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
   const float M = __ldcg(&tb.brk[row].M);
   int llo = __ldcg(&tb.brk[row].llo), lhi = __ldcg(&tb.brk[row].lhi);
 
-  // the candidate list, loaded whole in the same round as the records (its
-  // length is one of them); only the first ccnt entries are used
-  constexpr int kCPT = kCandCap / kTThreads;
-  unsigned long long cpre[kCPT];
+  // The candidate list (whole: its length is one of the records) and the
+  // segment's first block of kept-for-certain mask words go to shared memory
+  // asynchronously, in the same round as the records.
+  const int64_t seg_lo = (int64_t)r_first * p.rstages * 128;
+  const int64_t seg_hi = min(n, (int64_t)r_last * p.rstages * 128);
+  const int64_t mw_lo = seg_lo >> 5, mw_hi = (seg_hi + 31) >> 5;  // 4-word aligned
   {
     const unsigned long long* cand = tb.cand + row * kCandCap;
-#pragma unroll
-    for (int j = 0; j < kCPT; ++j) cpre[j] = __ldcg(cand + tid + j * kTThreads);
+    for (int i = tid; i < kCandCap / 2; i += kTThreads) cp_async16(&S.cand[2 * i], cand + 2 * i);
+    const uint32_t* hm = tb.hmask + row * tb.mask_words + mw_lo;
+    const int nw0 = (int)min((int64_t)kMaskBlock, mw_hi - mw_lo);
+    for (int i = tid; 4 * i < nw0; i += kTThreads) cp_async16(&S.mask0[4 * i], hm + 4 * i);
+    cp_async_commit();
   }
   // ---- 1. row totals (warp 0: one range record per lane) ----------------------
   if (warp == 0) {
@@ -306,32 +333,33 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
   const int m = fast ? (int)ccnt : 0;
   if (tid == 0) {
     S.found = 0;
-    S.okmin = 0xffffffffu;
-    S.okmax = 0u;
+    S.nlist = 0u;
   }
+  cp_async_wait<0>();
   __syncthreads();
+  // fast path: the segment's window keys (the candidates with an index in
+  // it) to a flat list, and the value rows of the first kVPre of them copied
+  // in while the cut is searched
+  unsigned long long* fl_key = &S.wl_key[0][0];  // flat list of kTWarps * kWList entries
   if (fast) {
-    // Every window key is a candidate, and the level is monotone in the
-    // logit, so a key lies in the window iff its order key lies between the
-    // candidates' lowest and highest.
-    uint32_t omin = 0xffffffffu, omax = 0u;
-#pragma unroll
-    for (int j = 0; j < kCPT; ++j) {
-      if (tid + j * kTThreads < m) {
-        S.cand[tid + j * kTThreads] = cpre[j];
-        const uint32_t ok = (uint32_t)(cpre[j] >> 32);
-        omin = min(omin, ok);
-        omax = max(omax, ok);
+    for (int i = tid; i < m; i += kTThreads) {
+      const unsigned long long ck = S.cand[i];
+      const uint32_t idx = 0xffffffffu - (uint32_t)(ck & 0xffffffffull);
+      if ((int64_t)idx >= seg_lo && (int64_t)idx < seg_hi) {
+        const uint32_t slot = atomicAdd(&S.nlist, 1u);
+        fl_key[slot] = ck;
       }
     }
-    omin = __reduce_min_sync(0xffffffffu, omin);
-    omax = __reduce_max_sync(0xffffffffu, omax);
-    if (lane == 0) {
-      atomicMin(&S.okmin, omin);
-      atomicMax(&S.okmax, omax);
+    __syncthreads();
+    const int npre = min((int)S.nlist, kVPre);
+    const __nv_bfloat16* Vr = V + (row / p.gm) * n * kTD;
+    for (int i = tid; i < npre * (kTD / 8); i += kTThreads) {  // 16 pieces of 16 B per row
+      const int e = i / (kTD / 8), c = i % (kTD / 8);
+      const uint32_t idx = 0xffffffffu - (uint32_t)(fl_key[e] & 0xffffffffull);
+      cp_async16(&S.vrow[e][2 * c], Vr + (int64_t)idx * kTD + 8 * c);
     }
+    cp_async_commit();
   }
-  __syncthreads();
 
   // ---- 2. the exact cut --------------------------------------------------------
   const long long nsub = 64ll * ((long long)lhi - (long long)llo);
@@ -587,30 +615,28 @@ full_sort:
       __syncthreads();
     }
     uint32_t pos_out = NHbefore + S.off_win;
-    const uint32_t wok_lo = S.okmin, wok_span = S.okmax - S.okmin;  // fast path only
     float ah[4] = {0.f, 0.f, 0.f, 0.f}, at[4] = {0.f, 0.f, 0.f, 0.f};
     double whw = 0.0, wtw = 0.0;
     float dmx = kNegInf;
-    int nl = 0;  // entries in this warp's window list (warp-uniform)
-    unsigned long long* wlk = S.wl_key[warp];
-    unsigned char* wlf = S.wl_kept[warp];
-    // value rows of the listed window keys, eight loads in flight per round
-    auto drain = [&]() {
-      for (int e0 = 0; e0 < nl; e0 += 8) {
+    // value rows of listed window keys: entries first, first + stride, ...
+    // below end, eight loads in flight per round (whole warp)
+    auto gather_list = [&](const unsigned long long* keys, const unsigned char* kept, int first,
+                           int end, int stride) {
+      for (int e0 = first; e0 < end; e0 += 8 * stride) {
         uint2 v[8];
         float w8[8];
         int kp[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const int e = e0 + q;
+          const int e = e0 + q * stride;
           kp[q] = -1;
           w8[q] = 0.0f;
           v[q] = make_uint2(0u, 0u);
-          if (e < nl) {
-            const unsigned long long lk = wlk[e];
+          if (e < end) {
+            const unsigned long long lk = keys[e];
             const float x = __uint_as_float((uint32_t)(lk >> 32));
             w8[q] = weight(x, M, sc);
-            kp[q] = wlf[e];
+            kp[q] = kept[e];
             v[q] = __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)(uint32_t)lk * kTD) + lane);
             if (!kp[q]) dmx = fmaxf(dmx, x);
           }
@@ -637,8 +663,113 @@ full_sort:
         }
       }
       __syncwarp();
-      nl = 0;
     };
+    if (fast) {
+      // The window keys of the segment are the candidates with an index in it
+      // (the flat list); every other key's side is in the value pass's
+      // kept-for-certain mask.  The first kVPre value rows are in shared memory.
+      const int nlist = (int)S.nlist;
+      cp_async_wait<0>();
+      __syncthreads();
+      for (int e0 = warp; e0 < nlist; e0 += 8 * kTWarps) {
+        uint2 v[8];
+        float w8[8];
+        int kp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = e0 + q * kTWarps;
+          kp[q] = -1;
+          w8[q] = 0.0f;
+          v[q] = make_uint2(0u, 0u);
+          if (e < nlist) {
+            const unsigned long long ck = fl_key[e];
+            const float x = ck_logit(ck);
+            const uint32_t idx = 0xffffffffu - (uint32_t)(ck & 0xffffffffull);
+            w8[q] = weight(x, M, sc);
+            kp[q] = ck >= cut ? 1 : 0;
+            v[q] = e < kVPre ? S.vrow[e][lane]
+                             : __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)idx * kTD) + lane);
+            if (!kp[q]) dmx = fmaxf(dmx, x);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (kp[q] < 0) continue;
+          const float2 a = bf16x2_to_float2(v[q].x), b = bf16x2_to_float2(v[q].y);
+          if (kp[q]) {
+            ah[0] = fmaf(w8[q], a.x, ah[0]);
+            ah[1] = fmaf(w8[q], a.y, ah[1]);
+            ah[2] = fmaf(w8[q], b.x, ah[2]);
+            ah[3] = fmaf(w8[q], b.y, ah[3]);
+            whw += (double)w8[q];
+          } else {
+            if constexpr (ERR) {
+              at[0] = fmaf(w8[q], a.x, at[0]);
+              at[1] = fmaf(w8[q], a.y, at[1]);
+              at[2] = fmaf(w8[q], b.x, at[2]);
+              at[3] = fmaf(w8[q], b.y, at[3]);
+            }
+            wtw += (double)w8[q];
+          }
+        }
+      }
+      // kept indices: mask words of the segment, in blocks of kMaskBlock words
+      const int64_t w_lo = mw_lo, w_hi = mw_hi;
+      const uint32_t* hm = tb.hmask + row * tb.mask_words;
+      for (int64_t wb0 = w_lo; wb0 < w_hi; wb0 += kMaskBlock) {
+        const int nwb = (int)min((int64_t)kMaskBlock, w_hi - wb0);
+        uint32_t kw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int wi = 4 * tid + j;
+          kw[j] = wi < nwb ? (wb0 == w_lo ? S.mask0[wi] : __ldcg(hm + wb0 + wi)) : 0u;
+          S.u.mk.win[wi] = 0u;
+        }
+        __syncthreads();
+        for (int e = tid; e < nlist; e += kTThreads) {  // the block's kept window keys
+          const unsigned long long ck = fl_key[e];
+          const uint32_t idx = 0xffffffffu - (uint32_t)(ck & 0xffffffffull);
+          const int64_t wi = ((int64_t)idx >> 5) - wb0;
+          if (ck >= cut && wi >= 0 && wi < nwb) atomicOr(&S.u.mk.win[wi], 1u << (idx & 31u));
+        }
+        __syncthreads();
+        uint32_t c = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          kw[j] |= S.u.mk.win[4 * tid + j];
+          c += __popc(kw[j]);
+        }
+        U128 dummy = u128_zero();
+        uint32_t ex = c;
+        block_excl_scan(dummy, ex, S);
+        uint32_t o = ex;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          S.u.mk.word[4 * tid + j] = kw[j];
+          S.u.mk.off[4 * tid + j] = o;
+          o += __popc(kw[j]);
+        }
+        if (tid == kTThreads - 1) S.off_win = o;  // the block's kept keys
+        __syncthreads();
+        // one 32-key word per warp step: coalesced index writes
+        for (int wi = warp; wi < nwb; wi += kTWarps) {
+          const uint32_t bits = S.u.mk.word[wi];
+          if ((bits >> lane) & 1u) {
+            const uint32_t at_ = pos_out + S.u.mk.off[wi] + __popc(bits & ((1u << lane) - 1u));
+            if (at_ < (uint32_t)n) dst[at_] = (int32_t)(((wb0 + wi) << 5) + lane);
+          }
+        }
+        pos_out += S.off_win;
+        __syncthreads();
+      }
+    } else {
+      int nl = 0;  // entries in this warp's window list (warp-uniform)
+      unsigned long long* wlk = S.wl_key[warp];
+      unsigned char* wlf = S.wl_kept[warp];
+      auto drain = [&]() {
+        gather_list(wlk, wlf, 0, nl, 1);
+        nl = 0;
+      };
     for (int64_t b0 = k_lo; b0 < k_hi; b0 += (int64_t)kBatch * kChunk) {
       float4 xv[kBatch];
 #pragma unroll
@@ -663,7 +794,7 @@ full_sort:
           // window lies on the side of the cut that its bracket side names)
           if (valid && (ok > cut_key || (ok == cut_key && (uint32_t)(key0 + e) <= cut_idx)))
             kbits |= 1u << (4 * c + e);
-          const bool win = fast ? (ok - wok_lo <= wok_span) : in_window(xs[e], sc, llo, lhi);
+          const bool win = in_window(xs[e], sc, llo, lhi);
           if (valid && win) wbits |= 1u << (4 * c + e);
         }
         pk[c >> 2] += (unsigned long long)__popc((kbits >> (4 * c)) & 0xfu) << (16 * (c & 3));
@@ -712,8 +843,8 @@ full_sort:
       }
       pos_out = chunk_base;
     }
-    if (nl) drain();
-
+      if (nl) drain();
+    }
     // ---- the range's results: value pass partial + window sums -------------------
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
