@@ -387,6 +387,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned b
       : "memory");
 }
 
+// Prefetch of global memory into L2 (a hint: no completion, no data returned).
+// src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Transposed butterfly reduction across the LPK lanes that share one key,
 // without selects.  Each lane holds CNT partial sums, slot s holding row

@@ -82,19 +82,34 @@ constexpr int kGBox = 64;             // dimensions per TMA box: 128 bytes of bf
 constexpr int kGV = kGK * kGD * 2;    // value bytes per stage (32 KB)
 constexpr int kGW = kGN * kGK * 2;    // weight-tile bytes per stage (8 KB)
 constexpr int kGU = 4 * kGK * 4;      // logit bytes per stage: up to four rows of kGK fp32 (2 KB)
-constexpr int kGWarps = 6;
+constexpr int kGWarps = 10;
 constexpr int kGThreads = kGWarps * kWarp;
 constexpr int kGWeightWarp0 = 2;
-constexpr int kGEpiThreads = 4 * kWarp;  // the four weight warps also read the accumulator
+constexpr int kGWeightWarps = 8;
+constexpr int kGEpiThreads = kGWeightWarps * kWarp;  // the weight warps also read the accumulator
 constexpr int kGEpiBar = 1;           // named barrier of the weight warps
 constexpr uint32_t kGTmemCols = 2 * kGN;
-constexpr int kCandBuf = 256;         // window keys a weight warp buffers (>= 128: one stage's)
-constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU) + 4 * kCandBuf * 8;
+constexpr int kCandBuf = 128;         // window keys a weight warp buffers (>= 128: one stage's)
+constexpr int kGPrefetch = 12;        // value stages per CTA prefetched into L2 beyond the ring
+constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU) + kGWeightWarps * kCandBuf * 8;
 static_assert(kGK % 64 == 0 && kGK <= 256, "a stage is whole 64-key swizzle atoms, one TMA box");
 static_assert(kGSmem <= 227 * 1024, "shared memory");
 
 constexpr int kMergeOct = 64;         // octaves of the merged per-row frame (two per lane)
 constexpr int kFineOctMax = 4;        // window octaves refined with the fine counts
+
+// A weight warp's part of a range record, handed to its partner warp.
+struct RecPart {
+  U128 mz, mh, mt;
+  double wh, wt;
+  uint32_t nh, nw;
+  float tmax;
+};
+
+__device__ __forceinline__ RowBracket ld_cg_bracket(const RowBracket* b) {
+  const int4 v = __ldcg(reinterpret_cast<const int4*>(b));
+  return RowBracket{__int_as_float(v.x), v.y, v.z, (uint32_t)v.w};
+}
 
 struct GItem {
   int tile, range, group;
@@ -172,86 +187,10 @@ __device__ __forceinline__ float warp_sum_f(float v) {
   return v;
 }
 
-// Fine counts of the window bins of 32 ranges r0 .. r0 + 31 (ranges >= nr
-// contribute nothing): lane l adds bins g0 + 2 NQ l ... g0 + 2 NQ l + 2 NQ - 1
-// of every range, two per 32-bit load, all loads of the round issued before
-// their sums (no branches: out-of-frame bins are loaded clamped and masked).
-template <int NQ>
-__device__ __forceinline__ void fine_round(const RangeHist* __restrict__ rh, int r0, int nr,
-                                           int my_sh, int g0, uint32_t* cnt) {
-  const int lane = threadIdx.x & 31;
-  constexpr int JC = NQ <= 2 ? 32 : 16;  // ranges per batch of loads (register budget)
-#pragma unroll
-  for (int j0 = 0; j0 < 32; j0 += JC) {
-    uint32_t w[JC][NQ];
-#pragma unroll
-    for (int j = 0; j < JC; ++j) {
-      const int sh = __shfl_sync(0xffffffffu, my_sh, j0 + j);
-      const RangeHist* h = rh + min(r0 + j0 + j, nr - 1);
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const int gi = g0 + 2 * NQ * lane + 2 * q + sh * kLevelsPerOctave;  // even
-        const bool ok = r0 + j0 + j < nr && gi >= 0 && gi + 1 < kHistBins;
-        const uint32_t v = __ldcg(reinterpret_cast<const unsigned int*>(
-            &h->fine[min(max(gi, 0), kHistBins - 2)]));
-        w[j][q] = ok ? v : 0u;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < JC; ++j) {
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        cnt[2 * q] += w[j][q] & 0xffffu;
-        cnt[2 * q + 1] += w[j][q] >> 16;
-      }
-    }
-  }
-}
-
-// Merges one round of 32 ranges into the row's merged octave sums mu (octaves
-// lane, lane + 32): range r's octave o is merged octave O = o - sh_r,
-// sh_r = (top_r - T) / 64; the headers of range r0 + lane are in this lane.
-__device__ __forceinline__ void merge_round(const RangeHist* __restrict__ rh, int nr, int T,
-                                            float p_delta, int r0, int my_top, uint32_t my_flags,
-                                            uint32_t my_below, const float (&oa)[32],
-                                            const float (&ob)[32], float (&mu)[2], float& deep,
-                                            bool& bad) {
-  const int lane = threadIdx.x & 31;
-  const bool mine = r0 + lane < nr;
-  bad |= mine && (my_flags != 0u || (my_top % kLevelsPerOctave) != 0);
-  const int my_sh = mine ? (my_top - T) / kLevelsPerOctave : 0;
-  // the range's keys below its own frame: fine index >= kHistBins - 64 sh
-  deep += mine ? (float)my_below * p_delta * pow2f_int(my_sh - kHistOctaves) : 0.0f;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int sh = __shfl_sync(0xffffffffu, my_sh, j);
-    const bool rj = r0 + j < nr;
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int o = lane + 32 * k + sh;  // the range octave that merged octave O needs
-      const float va = __shfl_sync(0xffffffffu, oa[j], o & 31);
-      const float vb = __shfl_sync(0xffffffffu, ob[j], o & 31);
-      mu[k] += (rj && o >= 0 && o < kHistOctaves) ? (o < 32 ? va : vb) : 0.0f;
-    }
-  }
-  // rare: ranges whose first stage lies so far below the row maximum that
-  // some of their octaves fall below the merged frame (sh <= -17)
-  const uint32_t far = __ballot_sync(0xffffffffu, mine && my_sh <= kHistOctaves - 1 - kMergeOct);
-  for (uint32_t f = far; f; f &= f - 1) {
-    const int j = __ffs(f) - 1;
-    const int sh = __shfl_sync(0xffffffffu, my_sh, j);
-    const RangeHist* h = rh + r0 + j;
-    for (int o = max(kMergeOct + sh, 0) + lane; o < kHistOctaves; o += 32) {
-      const uint32_t c = __ldcg(&h->ocnt[o]);
-      deep += (float)c * p_delta * pow2f_int(sh - o);
-    }
-  }
-}
-
-// The bracket of one row's cut, computed by one warp from the row's range
-// histograms and range maxima.  Returns (llo, lhi) through the references and
-// the row maximum M.  Every CTA that handles a range of the row computes the
-// same values from the same data, in the same order.
+// ---------------------------------------------------------------------------
+// The bracket of each row's cut: one CTA of kBWarps warps per row, between the
+// logits pass and the value pass.  Reads the row's range histograms and range
+// maxima and writes the row's RowBracket (M, llo, lhi).
 //
 // Frame: T = 64 ceil(X_M), X_M = fl(M * scale2), so every key's level is <= T;
 // merged fine index g = T - level, octave O = g / 64.  A key with fine index g
@@ -259,180 +198,281 @@ __device__ __forceinline__ void merge_round(const RangeHist* __restrict__ rh, in
 // i.e. 2^(delta - (g + 1)/64) <= w <= 2^(delta - g/64) up to the relative slack
 // s, where delta = T/64 - X_M in [0, 1) and E covers the fp32 rounding of
 // a = (M - u) * scale2 against X_M - x and exp2f's error; s also covers the
-// fp32 arithmetic of the bounds themselves (sums of at most ~3000 terms).
-// Every loop is branch-free and fully unrolled so that its loads and
-// shuffles overlap.
-__device__ void row_bracket(const RangeHist* __restrict__ hist, const float* __restrict__ cmax,
-                            int64_t row, const Plan& p, float& M_out, int& llo, int& lhi,
-                            unsigned long long* loads_done) {
+// fp32 arithmetic of the bounds themselves (sums of a few thousand terms in
+// any order).
+//
+// Steps: (1) every warp loads the headers and octave sums of its ranges
+// (range r to warp r % kBWarps, up to kBPre ranges per warp in flight) while
+// the block reduces the row maximum; (2) each warp merges its ranges into the
+// row frame (range r's octave o is merged octave o - sh_r, sh_r = (top_r - T)
+// / 64), the warps' partial sums are added in warp order; (3) warp 0 bounds the
+// mass below every octave boundary and finds the window octaves [Ohi, Olo);
+// (4) every warp adds its ranges' fine counts of the window bins into shared
+// counters (integers: order-free); (5) warp 0 refines the boundaries bin by bin.
+// ---------------------------------------------------------------------------
+constexpr int kBWarps = 8;
+constexpr int kBThreads = kBWarps * kWarp;
+constexpr int kBPre = 4;  // ranges per warp whose loads go out before the row maximum is known
+
+struct RangeHead {
+  int top;
+  uint32_t flags, below;
+  float oa, ob;  // octave sums o = lane and o = lane + 32 (0 past the frame)
+};
+
+__device__ __forceinline__ RangeHead load_head(const RangeHist* h) {
   const int lane = threadIdx.x & 31;
+  RangeHead x;
+  x.top = __ldcg(&h->top);
+  x.flags = __ldcg(&h->flags);
+  x.below = __ldcg(&h->below);
+  x.oa = __ldcg(&h->omass[lane]);
+  x.ob = lane + 32 < kHistOctaves ? __ldcg(&h->omass[lane + 32]) : 0.0f;
+  return x;
+}
+
+// Adds one range to the warp's merged octave sums mu (octaves lane, lane + 32)
+// and its deep mass (keys below the merged frame; summed on lane 0 only for
+// the range's own below-frame count).
+__device__ __forceinline__ void merge_range(const RangeHist* h, const RangeHead& x, int T,
+                                            float p_delta, float (&mu)[2], float& deep, bool& bad) {
+  const int lane = threadIdx.x & 31;
+  bad |= x.flags != 0u || (x.top % kLevelsPerOctave) != 0;
+  const int sh = (x.top - T) / kLevelsPerOctave;
+  if (lane == 0) deep += (float)x.below * p_delta * pow2f_int(sh - kHistOctaves);
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int o = lane + 32 * k + sh;  // the range octave that merged octave O needs
+    const float va = __shfl_sync(0xffffffffu, x.oa, o & 31);
+    const float vb = __shfl_sync(0xffffffffu, x.ob, o & 31);
+    mu[k] += (o >= 0 && o < kHistOctaves) ? (o < 32 ? va : vb) : 0.0f;
+  }
+  // rare: the range's frame reaches below the merged frame (sh <= -17)
+  if (sh <= kHistOctaves - 1 - kMergeOct) {
+    for (int o = max(kMergeOct + sh, 0) + lane; o < kHistOctaves; o += 32)
+      deep += (float)__ldcg(&h->ocnt[o]) * p_delta * pow2f_int(sh - o);
+  }
+}
+
+// Adds one range's fine counts of the window bins: lane l covers bin pairs
+// 64 q + 2 l (q < nwo) of the window that starts at merged fine index g0.
+__device__ __forceinline__ void fine_range(const RangeHist* h, int sh, int g0, int nwo,
+                                           uint32_t (&c)[2 * kFineOctMax]) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v[kFineOctMax];
+#pragma unroll
+  for (int q = 0; q < kFineOctMax; ++q) {
+    const int gi = g0 + kLevelsPerOctave * q + 2 * lane + sh * kLevelsPerOctave;  // even
+    const bool ok = q < nwo && gi >= 0 && gi + 1 < kHistBins;
+    v[q] = ok ? __ldcg(reinterpret_cast<const unsigned int*>(&h->fine[gi])) : 0u;
+  }
+#pragma unroll
+  for (int q = 0; q < kFineOctMax; ++q) {
+    c[2 * q] += v[q] & 0xffffu;
+    c[2 * q + 1] += v[q] >> 16;
+  }
+}
+
+__global__ void __launch_bounds__(kBThreads)
+bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ cmax,
+                  RowBracket* __restrict__ brk, Plan p) {
+  // the histograms and maxima are complete; the value pass may be scheduled
+  // from here on (after the logits pass, and so after the caller's kernels)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ float s_mu[kBWarps][kMergeOct];
+  __shared__ float s_deep[kBWarps], s_max[kBWarps];
+  __shared__ uint32_t s_cnt[kFineOctMax * kLevelsPerOctave];
+  __shared__ int s_olo, s_ohi;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t row = blockIdx.x;
   const int nr = p.nranges;
   const RangeHist* rh = hist + row * nr;
-  // lane 0 signals (once) when the bracket's loads no longer wait behind the value stream
-  bool signalled = loads_done == nullptr;
-  auto signal = [&]() {
-    if (!signalled && lane == 0) mbar_arrive(loads_done);
-    signalled = true;
-  };
-  // Round 0 of the loads, all issued before any is used: the range maxima, the
-  // headers and the octave sums of ranges 0 .. 31 (octave o in lane o % 32).
-  const int rl0 = min(lane, nr - 1);
-  float M = __ldcg(cmax + row * p.nchunks + rl0);
-  const int top0 = __ldcg(&rh[rl0].top);
-  const uint32_t flags0 = __ldcg(&rh[rl0].flags);
-  const uint32_t below0 = __ldcg(&rh[rl0].below);
-  float oa0[32], ob0[32];
+  for (int i = threadIdx.x; i < kFineOctMax * kLevelsPerOctave; i += kBThreads) s_cnt[i] = 0u;
+
+  // (1) loads of the first kBPre ranges of this warp, and the row maximum
+  RangeHead pre[kBPre];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const RangeHist* h = rh + min(j, nr - 1);
-    oa0[j] = __ldcg(&h->omass[lane]);
-    ob0[j] = __ldcg(&h->omass[min(lane + 32, kHistOctaves - 1)]);
-  }
-  for (int r = 32 + lane; r < nr; r += 32) M = fmaxf(M, __ldcg(cmax + row * p.nchunks + r));
+  for (int i = 0; i < kBPre; ++i) pre[i] = load_head(rh + min(warp + kBWarps * i, nr - 1));
+  float M = kNegInf;
+  for (int r = threadIdx.x; r < nr; r += kBThreads) M = fmaxf(M, __ldcg(cmax + row * p.nchunks + r));
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  M_out = M;
-  llo = INT_MIN;  // defaults: every key is in the window
-  lhi = INT_MAX;
+  if (lane == 0) s_max[warp] = M;
+  __syncthreads();
+  M = s_max[0];
+#pragma unroll
+  for (int w = 1; w < kBWarps; ++w) M = fmaxf(M, s_max[w]);
+  RowBracket out{M, INT_MIN, INT_MAX, 0u};  // default: every key is in the window
   const float XM = __fmul_rn(M, p.scale2);
   if (!(fabsf(XM) < 1.0e6f)) {  // non-finite rows: flagged by the logits pass
-    signal();
+    if (threadIdx.x == 0) brk[row] = out;
     return;
   }
   const int T = __float2int_ru(XM) * kLevelsPerOctave;
   const float delta = (float)((double)T / kLevelsPerOctave - (double)XM);  // in [0, 1)
   const float p_delta = exp2f(delta);
-  const float p_64 = exp2f(-1.0f / kLevelsPerOctave);
-  const float slack = (fabsf(XM) + 2.0f * kMergeOct + 64.0f) * 0x1p-22f + 1.0e-4f;
 
-  // coarse merge: octaves O = lane and lane + 32 of the merged frame
+  // (2) merge this warp's ranges in range order
   bool bad = false;
   float mu[2] = {0.0f, 0.0f};
   float deep = 0.0f;  // upper bound of the mass of keys below the merged frame
-  merge_round(rh, nr, T, p_delta, 0, top0, flags0, below0, oa0, ob0, mu, deep, bad);
-  for (int r0 = 32; r0 < nr; r0 += 32) {  // more than 32 ranges per row (large n)
-    const int rl = min(r0 + lane, nr - 1);
-    const int my_top = __ldcg(&rh[rl].top);
-    const uint32_t my_flags = __ldcg(&rh[rl].flags), my_below = __ldcg(&rh[rl].below);
-    float oa[32], ob[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const RangeHist* h = rh + min(r0 + j, nr - 1);
-      oa[j] = __ldcg(&h->omass[lane]);
-      ob[j] = __ldcg(&h->omass[min(lane + 32, kHistOctaves - 1)]);
-    }
-    merge_round(rh, nr, T, p_delta, r0, my_top, my_flags, my_below, oa, ob, mu, deep, bad);
+  for (int i = 0; i < kBPre; ++i) {
+    const int r = warp + kBWarps * i;
+    if (r < nr) merge_range(rh + r, pre[i], T, p_delta, mu, deep, bad);
   }
-  if (__any_sync(0xffffffffu, bad)) {
-    signal();
+  for (int r = warp + kBWarps * kBPre; r < nr; r += kBWarps)  // many ranges (large n)
+    merge_range(rh + r, load_head(rh + r), T, p_delta, mu, deep, bad);
+  s_mu[warp][lane] = mu[0];
+  s_mu[warp][lane + 32] = mu[1];
+  deep = warp_sum_f(deep);
+  if (lane == 0) s_deep[warp] = deep;
+  if (__syncthreads_or(bad)) {
+    if (threadIdx.x == 0) brk[row] = out;
     return;
   }
-  deep = warp_sum_f(deep) * (1.0f + slack);
-  // per-octave mass bounds; octave O holds weights 2^(delta - O - j/64) per unit of omass
-  float hi_m[2], lo_m[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const float f = p_delta * pow2f_int(-(lane + 32 * k));
-    hi_m[k] = mu[k] * f * (1.0f + slack);
-    lo_m[k] = mu[k] * f * p_64 * (1.0f - slack);
-  }
-  // suffix sums from the bottom of the frame: mass of octaves >= O
-  const float upU = warp_suffix_sum_f(hi_m[1]), upL = warp_suffix_sum_f(lo_m[1]);
-  const float totU1 = __shfl_sync(0xffffffffu, upU, 0), totL1 = __shfl_sync(0xffffffffu, upL, 0);
-  const float loU = warp_suffix_sum_f(hi_m[0]) + totU1, loL = warp_suffix_sum_f(lo_m[0]) + totL1;
-  const float ZU = __shfl_sync(0xffffffffu, loU, 0) + deep;
-  const float ZL = __shfl_sync(0xffffffffu, loL, 0);
+
+  // (3) warp 0: octave bounds and the window octaves
+  const float slack = (fabsf(XM) + 2.0f * kMergeOct + 64.0f) * 0x1p-22f + 1.0e-4f;
+  const float p_64 = exp2f(-1.0f / kLevelsPerOctave);
   const float eps = (float)p.eps;
-  // D+(O) <= eps ZL: the keys of octaves >= O are certainly dropped
-  // D-(O) >  eps ZU: the keys of octaves <  O are certainly kept
-  const uint32_t tail0 = __ballot_sync(0xffffffffu, loU + deep <= eps * ZL);
-  const uint32_t tail1 = __ballot_sync(0xffffffffu, upU + deep <= eps * ZL);
-  const uint32_t head0 = __ballot_sync(0xffffffffu, loL > eps * ZU);
-  const uint32_t head1 = __ballot_sync(0xffffffffu, upL > eps * ZU);
-  // smallest O with the tail condition (kMergeOct: only the deep keys;
-  // kMergeOct + 1: none), largest O with the head condition (0 if none)
-  const int Olo = tail0 ? __ffs(tail0) - 1 : tail1 ? 32 + __ffs(tail1) - 1
-                : (deep <= eps * ZL ? kMergeOct : kMergeOct + 1);
-  const int Ohi = head1 ? 32 + 31 - __clz(head1) : head0 ? 31 - __clz(head0) : 0;
+  float loU = 0.0f, loL = 0.0f, upU = 0.0f, upL = 0.0f, ZU = 0.0f, ZL = 0.0f;
+  int Olo = 0, Ohi = 0;
+  if (warp == 0) {
+    mu[0] = s_mu[0][lane];
+    mu[1] = s_mu[0][lane + 32];
+    deep = s_deep[0];
+#pragma unroll
+    for (int w = 1; w < kBWarps; ++w) {
+      mu[0] += s_mu[w][lane];
+      mu[1] += s_mu[w][lane + 32];
+      deep += s_deep[w];
+    }
+    deep *= 1.0f + slack;
+    // per-octave mass bounds; octave O holds weights 2^(delta - O - j/64) per unit of omass
+    float hi_m[2], lo_m[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float f = p_delta * pow2f_int(-(lane + 32 * k));
+      hi_m[k] = mu[k] * f * (1.0f + slack);
+      lo_m[k] = mu[k] * f * p_64 * (1.0f - slack);
+    }
+    // suffix sums from the bottom of the frame: mass of octaves >= O
+    upU = warp_suffix_sum_f(hi_m[1]);
+    upL = warp_suffix_sum_f(lo_m[1]);
+    const float totU1 = __shfl_sync(0xffffffffu, upU, 0), totL1 = __shfl_sync(0xffffffffu, upL, 0);
+    loU = warp_suffix_sum_f(hi_m[0]) + totU1;
+    loL = warp_suffix_sum_f(lo_m[0]) + totL1;
+    ZU = __shfl_sync(0xffffffffu, loU, 0) + deep;
+    ZL = __shfl_sync(0xffffffffu, loL, 0);
+    // D+(O) <= eps ZL: the keys of octaves >= O are certainly dropped
+    // D-(O) >  eps ZU: the keys of octaves <  O are certainly kept
+    const uint32_t tail0 = __ballot_sync(0xffffffffu, loU + deep <= eps * ZL);
+    const uint32_t tail1 = __ballot_sync(0xffffffffu, upU + deep <= eps * ZL);
+    const uint32_t head0 = __ballot_sync(0xffffffffu, loL > eps * ZU);
+    const uint32_t head1 = __ballot_sync(0xffffffffu, upL > eps * ZU);
+    // smallest O with the tail condition (kMergeOct: only the deep keys;
+    // kMergeOct + 1: none), largest O with the head condition (0 if none)
+    Olo = tail0 ? __ffs(tail0) - 1 : tail1 ? 32 + __ffs(tail1) - 1
+          : (deep <= eps * ZL ? kMergeOct : kMergeOct + 1);
+    Ohi = head1 ? 32 + 31 - __clz(head1) : head0 ? 31 - __clz(head0) : 0;
+    if (lane == 0) {
+      s_olo = Olo;
+      s_ohi = Ohi;
+    }
+  }
+  __syncthreads();
+  Olo = s_olo;
+  Ohi = s_ohi;
   if (Olo <= Ohi) {  // cannot happen with consistent bounds; keep the default
-    signal();
+    if (threadIdx.x == 0) brk[row] = out;
     return;
   }
   int g_lo = kLevelsPerOctave * Olo, g_hi = kLevelsPerOctave * Ohi;  // the coarse result
-  // fine refinement of the window octaves [Ohi, Olo)
   const int nwo = Olo - Ohi;
-  if (Olo <= kMergeOct && nwo <= kFineOctMax) {
-    // lane l owns the B = 2 nwo consecutive fine bins g0 + B l ... g0 + B l + B - 1
-    const int B = 2 * nwo;
+  const bool fine = Olo <= kMergeOct && nwo <= kFineOctMax;
+  if (fine) {
+    // (4) fine counts of the window bins [g0, g0 + 64 nwo)
     const int g0 = kLevelsPerOctave * Ohi;
-    uint32_t cnt[2 * kFineOctMax];
+    uint32_t c[2 * kFineOctMax];
 #pragma unroll
-    for (int b = 0; b < 2 * kFineOctMax; ++b) cnt[b] = 0u;
-    for (int r0 = 0; r0 < nr; r0 += 32) {
-      const int my_sh =
-          ((r0 == 0 ? top0 : __ldcg(&rh[min(r0 + lane, nr - 1)].top)) - T) / kLevelsPerOctave;
-      switch (nwo) {
-        case 1: fine_round<1>(rh, r0, nr, my_sh, g0, cnt); break;
-        case 2: fine_round<2>(rh, r0, nr, my_sh, g0, cnt); break;
-        case 3: fine_round<3>(rh, r0, nr, my_sh, g0, cnt); break;
-        default: fine_round<4>(rh, r0, nr, my_sh, g0, cnt); break;
+    for (int b = 0; b < 2 * kFineOctMax; ++b) c[b] = 0u;
+#pragma unroll
+    for (int i = 0; i < kBPre; ++i) {
+      const int r = warp + kBWarps * i;
+      if (r < nr) fine_range(rh + r, (pre[i].top - T) / kLevelsPerOctave, g0, nwo, c);
+    }
+    for (int r = warp + kBWarps * kBPre; r < nr; r += kBWarps)
+      fine_range(rh + r, (__ldcg(&rh[r].top) - T) / kLevelsPerOctave, g0, nwo, c);
+#pragma unroll
+    for (int q = 0; q < kFineOctMax; ++q) {
+      if (q < nwo) {
+        if (c[2 * q]) atomicAdd(&s_cnt[kLevelsPerOctave * q + 2 * lane], c[2 * q]);
+        if (c[2 * q + 1]) atomicAdd(&s_cnt[kLevelsPerOctave * q + 2 * lane + 1], c[2 * q + 1]);
       }
     }
-    signal();
-    // per-bin bounds and suffix sums inside the window (bins below it: D(Olo))
-    const float baseU =
-        (Olo < kMergeOct ? __shfl_sync(0xffffffffu, (Olo < 32 ? loU : upU), Olo & 31) : 0.0f) + deep;
-    const float baseL =
-        (Olo < kMergeOct) ? __shfl_sync(0xffffffffu, (Olo < 32 ? loL : upL), Olo & 31) : 0.0f;
-    float bu[2 * kFineOctMax], bl[2 * kFineOctMax], su = 0.0f, sl = 0.0f;
+    __syncthreads();
+    if (warp == 0) {
+      // (5) lane l owns the B = 2 nwo consecutive window bins B l ... B l + B - 1
+      const int B = 2 * nwo;
+      const float baseU =
+          (Olo < kMergeOct ? __shfl_sync(0xffffffffu, (Olo < 32 ? loU : upU), Olo & 31) : 0.0f) + deep;
+      const float baseL =
+          (Olo < kMergeOct) ? __shfl_sync(0xffffffffu, (Olo < 32 ? loL : upL), Olo & 31) : 0.0f;
+      float bu[2 * kFineOctMax], bl[2 * kFineOctMax], su = 0.0f, sl = 0.0f;
 #pragma unroll
-    for (int b = 0; b < 2 * kFineOctMax; ++b) {
-      const int g = g0 + B * lane + b;
-      const float f = p_delta *
-                      exp2f(-(float)(g & (kLevelsPerOctave - 1)) / (float)kLevelsPerOctave) *
-                      pow2f_int(-(g / kLevelsPerOctave));
-      bu[b] = (b < B) ? (float)cnt[b] * f * (1.0f + slack) : 0.0f;
-      bl[b] = (b < B) ? (float)cnt[b] * f * p_64 * (1.0f - slack) : 0.0f;
-      su += bu[b];
-      sl += bl[b];
-    }
-    // mass of the window bins of the lanes above this one (larger g)
-    const float aboveU = warp_suffix_sum_f(su) - su, aboveL = warp_suffix_sum_f(sl) - sl;
-    // walk this lane's bins from its bottom (largest g) up
-    float DU = baseU + aboveU, DL = baseL + aboveL;
-    int my_lo = INT_MAX, my_hi = -1;
+      for (int b = 0; b < 2 * kFineOctMax; ++b) {
+        const int g = g0 + B * lane + b;
+        const float cnt = (b < B) ? (float)s_cnt[B * lane + b] : 0.0f;
+        const float f = p_delta *
+                        exp2f(-(float)(g & (kLevelsPerOctave - 1)) / (float)kLevelsPerOctave) *
+                        pow2f_int(-(g / kLevelsPerOctave));
+        bu[b] = cnt * f * (1.0f + slack);
+        bl[b] = cnt * f * p_64 * (1.0f - slack);
+        su += bu[b];
+        sl += bl[b];
+      }
+      // mass of the window bins of the lanes above this one (larger g)
+      const float aboveU = warp_suffix_sum_f(su) - su, aboveL = warp_suffix_sum_f(sl) - sl;
+      // walk this lane's bins from its bottom (largest g) up
+      float DU = baseU + aboveU, DL = baseL + aboveL;
+      int my_lo = INT_MAX, my_hi = -1;
 #pragma unroll
-    for (int b = 2 * kFineOctMax - 1; b >= 0; --b) {
-      DU += bu[b];
-      DL += bl[b];
-      const int g = g0 + B * lane + b;  // boundary at the top of bin g: keys with index >= g
-      const bool in = b < B;
-      my_lo = (in && DU <= eps * ZL) ? g : my_lo;
-      my_hi = (in && DL > eps * ZU && my_hi < 0) ? g : my_hi;
-    }
+      for (int b = 2 * kFineOctMax - 1; b >= 0; --b) {
+        DU += bu[b];
+        DL += bl[b];
+        const int g = g0 + B * lane + b;  // boundary at the top of bin g: keys with index >= g
+        const bool in = b < B;
+        my_lo = (in && DU <= eps * ZL) ? g : my_lo;
+        my_hi = (in && DL > eps * ZU && my_hi < 0) ? g : my_hi;
+      }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      my_lo = min(my_lo, __shfl_xor_sync(0xffffffffu, my_lo, o));
-      my_hi = max(my_hi, __shfl_xor_sync(0xffffffffu, my_hi, o));
-    }
-    if (my_lo != INT_MAX) g_lo = min(g_lo, my_lo);
-    if (my_hi >= 0) g_hi = max(g_hi, my_hi);
-    if (g_lo <= g_hi) {  // inconsistent: fall back to the coarse window
-      g_lo = kLevelsPerOctave * Olo;
-      g_hi = kLevelsPerOctave * Ohi;
+      for (int o = 16; o >= 1; o >>= 1) {
+        my_lo = min(my_lo, __shfl_xor_sync(0xffffffffu, my_lo, o));
+        my_hi = max(my_hi, __shfl_xor_sync(0xffffffffu, my_hi, o));
+      }
+      if (my_lo != INT_MAX) g_lo = min(g_lo, my_lo);
+      if (my_hi >= 0) g_hi = max(g_hi, my_hi);
+      if (g_lo <= g_hi) {  // inconsistent: fall back to the coarse window
+        g_lo = kLevelsPerOctave * Olo;
+        g_hi = kLevelsPerOctave * Ohi;
+      }
     }
   }
-  signal();
   // keys with fine index >= g_lo (level <= T - g_lo) are dropped, keys with
   // fine index < g_hi (level > T - g_hi) are kept
-  llo = (Olo > kMergeOct) ? INT_MIN : T - g_lo + 1;
-  lhi = T - g_hi + 1;
+  if (threadIdx.x == 0) {
+    out.llo = (Olo > kMergeOct) ? INT_MIN : T - g_lo + 1;
+    out.lhi = T - g_hi + 1;
+    brk[row] = out;
+  }
 }
 
 template <int RT, bool ERR>
 __global__ void __launch_bounds__(kGThreads, 1)
 gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restrict__ u,
-                 const float* __restrict__ cmax, TcBufs tb, float* __restrict__ acc_out, Plan p,
+                 const unsigned char* __restrict__ vbase, TcBufs tb, float* __restrict__ acc_out, Plan p,
                  uint32_t* __restrict__ status) {
   // the last kernel may be scheduled now; it waits for this grid
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -443,11 +483,14 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
   unsigned char* wring = base + kGStages * kGV;         // [kGStages][kGK / 64][kGN rows][128 B]
   float* uring = reinterpret_cast<float*>(wring + kGStages * kGW);  // [kGStages][4 rows][kGK]
   unsigned long long* cbuf_all =
-      reinterpret_cast<unsigned long long*>(uring + kGStages * 4 * kGK);  // [4][kCandBuf]
-  __shared__ unsigned long long vfull[kGStages], ufull[kGStages], wfull[kGStages], empty[kGStages];
+      reinterpret_cast<unsigned long long*>(uring + kGStages * 4 * kGK);  // [8][kCandBuf]
+  __shared__ unsigned long long vfull[kGStages], wfull[kGStages], empty[kGStages];
+  // the logits of stage t land on ufull[t % 2][t % kGStages]: each of these
+  // barriers serves one parity of stages, whose weight warps alone wait on it
+  // and see every one of its phases (a parity wait is sound only then)
+  __shared__ unsigned long long ufull[2][kGStages];
   __shared__ unsigned long long accfull[2], accempty[2], drain;
-  // the first item's bracket loads have returned: the value stream may start
-  __shared__ unsigned long long brk_loads;
+  __shared__ RecPart rpart[2][4];  // by item parity and row
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
 
@@ -464,7 +507,8 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGStages; ++s) {
       mbar_init(&vfull[s], 1);
-      mbar_init(&ufull[s], 1);
+      mbar_init(&ufull[0][s], 1);
+      mbar_init(&ufull[1][s], 1);
       mbar_init(&wfull[s], RT);
       mbar_init(&empty[s], 1);
     }
@@ -473,7 +517,6 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       mbar_init(&accempty[b], kGEpiThreads);
     }
     mbar_init(&drain, 1);
-    mbar_init(&brk_loads, 4);  // one arrival per weight warp
     s_abort = 0;
     mbar_fence_init();
   }
@@ -489,19 +532,25 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       const unsigned long long pol_u = policy_evict_last();  // read again by the last kernel
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(&vmap))
                    : "memory");
-      // The first ring of value stages goes out before the logits exist, once
-      // the weight warps' bracket loads are back: the flood of value loads
-      // would otherwise stretch their latency (bounded wait, then go anyway).
-      mbar_wait(&brk_loads, 0u);
-      int nA = 0;
-      for (int it = blockIdx.x; it < nitems && nA < kGStages; it += gridDim.x) {
+      // The first ring of value stages goes out at once (the value rows do not
+      // depend on the earlier kernels of the call), and the next kGPrefetch
+      // stages are prefetched into L2 while the brackets are computed.
+      int nA = 0, nP = 0;
+      for (int it = blockIdx.x; it < nitems && nP < kGStages + kGPrefetch; it += gridDim.x) {
         const GItem g = gitem_of(it, p);
         const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
-        for (int sg = s_lo; sg < s_hi && nA < kGStages; ++sg, ++nA) {
-          unsigned char* dst = vring + nA * kGV;
-          mbar_arrive_expect_tx(&vfull[nA], (unsigned)kGV);
-          tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[nA], pol);
-          tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[nA], pol);
+        for (int sg = s_lo; sg < s_hi && nP < kGStages + kGPrefetch; ++sg, ++nP) {
+          if (nA < kGStages) {
+            unsigned char* dst = vring + nA * kGV;
+            mbar_arrive_expect_tx(&vfull[nA], (unsigned)kGV);
+            tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[nA], pol);
+            tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[nA], pol);
+            ++nA;
+          } else {
+            const int64_t key0 = (int64_t)sg * kGK;
+            const unsigned bytes = (unsigned)min((int64_t)kGK, p.n - key0) * (unsigned)(kGD * 2);
+            bulk_prefetch_l2(vbase + ((int64_t)g.group * p.n + key0) * (kGD * 2), bytes);
+          }
         }
       }
       asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits pass has completed
@@ -528,10 +577,11 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
           // (the logit rows are padded to a multiple of 64 keys)
           const int64_t key0 = (int64_t)sg * kGK;
           const unsigned ub = (unsigned)((min((int64_t)kGK, p.n - key0) + 3) / 4) * 16u;
-          mbar_arrive_expect_tx(&ufull[slot], ub * (unsigned)nrows);
+          unsigned long long* ub_bar = &ufull[t & 1][slot];
+          mbar_arrive_expect_tx(ub_bar, ub * (unsigned)nrows);
           for (int r = 0; r < nrows; ++r)
             bulk_load(uring + (slot * 4 + r) * kGK, u + (row0 + r) * p.ustride + key0, ub,
-                      &ufull[slot], pol_u);
+                      ub_bar, pol_u);
         }
       }
       if (!ok) {
@@ -540,7 +590,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
         // the copies still in flight land before the CTA may exit (bounded)
         for (int t2 = max(0, t - kGStages); t2 < t; ++t2) {
           mbar_wait(&vfull[t2 % kGStages], (unsigned)(t2 / kGStages) & 1u);
-          mbar_wait(&ufull[t2 % kGStages], (unsigned)(t2 / kGStages) & 1u);
+          mbar_wait(&ufull[t2 & 1][t2 % kGStages], (unsigned)(t2 / (2 * kGStages)) & 1u);
         }
         for (int t2 = t; t2 < nA; ++t2) mbar_wait(&vfull[t2], 0u);
       }
@@ -588,194 +638,199 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       mbar_wait(&drain, 0u);
     }
   } else {
-    // ---------------- weights: warp r -> row r of the tile; accumulator ----------------
-    const int r = warp - kGWeightWarp0;
-    // warps without a row in the first item let the value stream start at once
-    const bool first_row = r < RT && blockIdx.x < nitems &&
-                           r < min(RT, p.gm - gitem_of(blockIdx.x, p).tile * RT);
-    if (!first_row && lane == 0) mbar_arrive(&brk_loads);
-    const int quarter = warp & 3;  // TMEM lanes (dimensions) this warp may read
+    // ---------------- weights (warps 2-9) and the accumulator ----------------
+    // warp wi = warp - 2 serves row r = wi % 4 of the tile in the stages t of
+    // parity h = wi / 4 (t counts the CTA's stages), so that two stages are in
+    // the works at once; it reads tensor-memory lanes 32 (warp % 4) ... + 31.
+    const int wi = warp - kGWeightWarp0;
+    const int r = wi & 3, h = wi >> 2;
+    const int quarter = warp & 3;
     const int dim = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    {
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // histograms and maxima are complete
-      const float sc = p.scale2;
-      int t = 0, jj = 0;
-      bool ok = true;
-      for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++jj) {
-        const GItem g = gitem_of(it, p);
-        const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
-        const int64_t row = (int64_t)g.group * p.gm + (int64_t)g.tile * RT + r;
-        const int nrows = min(RT, p.gm - g.tile * RT);
-        const bool row_ok = r < nrows;
-        float M = 0.0f;
-        int llo = INT_MIN, lhi = INT_MAX;
-        if (row_ok) {
-          row_bracket(tb.hist, cmax, row, p, M, llo, lhi,
-                      it == (int)blockIdx.x ? &brk_loads : nullptr);
-          if (g.range == 0 && lane == 0) tb.brk[row] = RowBracket{M, llo, lhi, 0u};
-        }
-        U128 mz = u128_zero(), mh = u128_zero(), mt = u128_zero();
-        double wh = 0.0, wt = 0.0;  // fp64 sums of per-stage fp32 weight sums (for KL only)
-        uint32_t nh = 0u, nw = 0u;
-        float tmax = kNegInf;
-        unsigned long long* cand = tb.cand + row * kCandCap;
-        unsigned long long* cbuf = cbuf_all + r * kCandBuf;
-        uint32_t nbuf = 0u;
-        for (int sg = s_lo; sg < s_hi && r < RT && ok; ++sg, ++t) {
-          const int slot = t % kGStages;
-          const int64_t k0 = (int64_t)sg * kGK + 4 * lane;  // this lane's four keys
-          // the stage's logits have landed; its slot's W tile is then free too
-          // (the MMAs that last read the slot have finished)
-          if (!mbar_wait(&ufull[slot], (unsigned)(t / kGStages) & 1u) || aborted(&s_abort)) ok = false;
-          if (!__all_sync(0xffffffffu, ok)) {
-            ok = false;
-            break;
-          }
-          float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (row_ok) x = reinterpret_cast<const float4*>(uring + (slot * 4 + r) * kGK)[lane];
-          uint32_t hp[4][3], tp[4][3];
-          const float xs[4] = {x.x, x.y, x.z, x.w};
-          uint32_t winmask = 0u, hbits = 0u;
-          float sh_ = 0.0f, st_ = 0.0f;
-          // branch-free: every key is kept (level >= lhi), dropped (< llo) or window
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const bool valid = row_ok && k0 + i < p.n;
-            const float w = valid ? weight(xs[i], M, sc) : 0.0f;
-            const int L = key_level(xs[i], sc);
-            const bool head = valid && L >= lhi;
-            const bool tail = valid && L < llo;
-            const unsigned long long W = mass62(w);
-            u128_add(mz, W);
-            u128_add(mh, head ? W : 0ull);
-            u128_add(mt, tail ? W : 0ull);
-            nh += head ? 1u : 0u;
-            hbits |= head ? (1u << i) : 0u;
-            nw += (valid && !head && !tail) ? 1u : 0u;
-            winmask |= (valid && !head && !tail) ? (1u << i) : 0u;
-            sh_ += head ? w : 0.0f;
-            st_ += tail ? w : 0.0f;
-            tmax = fmaxf(tmax, tail ? xs[i] : kNegInf);
-            uint32_t pt[3];
-            split3(w, pt);
-#pragma unroll
-            for (int part = 0; part < 3; ++part) {
-              hp[i][part] = head ? pt[part] : 0u;
-              if constexpr (ERR) tp[i][part] = tail ? pt[part] : 0u;
-            }
-          }
-          wh += (double)sh_;
-          wt += (double)st_;
-          // the stage's kept-for-certain bits: lane l holds keys 4 l .. 4 l + 3,
-          // i.e. bits 4 (l % 8) .. of word l / 8; eight lanes OR their nibbles
-          {
-            uint32_t wv = hbits << (4 * (lane & 7));
-            wv |= __shfl_xor_sync(0xffffffffu, wv, 1);
-            wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
-            wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
-            if (row_ok && (lane & 7) == 0) tb.hmask[row * tb.mask_words + 4 * (int64_t)sg + (lane >> 3)] = wv;
-          }
-          unsigned char* wtile = wring + slot * kGW;
-          const int c = lane >> 1;  // 16-byte piece (8 keys) along K; this lane writes one half
-          const uint32_t half = (uint32_t)(lane & 1) * 8u;
-#pragma unroll
-          for (int part = 0; part < 3; ++part) {
-            *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(0, part, r), c, kGN) + half) =
-                make_uint2(hp[0][part] | (hp[1][part] << 16), hp[2][part] | (hp[3][part] << 16));
-            if constexpr (ERR)
-              *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(1, part, r), c, kGN) + half) =
-                  make_uint2(tp[0][part] | (tp[1][part] << 16), tp[2][part] | (tp[3][part] << 16));
-          }
-          fence_proxy_async();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&wfull[slot]);
-          // window keys to this warp's buffer (flushed to the row's list when
-          // full and at the end of the item: one global atomic per flush)
-          if (__any_sync(0xffffffffu, winmask != 0u)) {
-            const uint32_t cnt = __popc(winmask);
-            uint32_t pre = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
-              if (lane >= o) pre += y;
-            }
-            const uint32_t total = __shfl_sync(0xffffffffu, pre, 31);
-            if (nbuf + total > (uint32_t)kCandBuf) {
-              flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
-              nbuf = 0u;
-            }
-            uint32_t at = nbuf + pre - cnt;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (winmask & (1u << i)) cbuf[at++] = composite(order_key(xs[i]), (uint32_t)(k0 + i));
-            }
-            __syncwarp();
-            nbuf += total;  // a stage adds at most 128 <= kCandBuf keys
-          }
-        }
-        if (row_ok && __any_sync(0xffffffffu, nbuf > 0u)) {
-          flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
-          nbuf = 0u;
-        }
-        if (ok) {
-          // the range record of this row
-          mz = u128_warp_sum(mz);
-          mh = u128_warp_sum(mh);
-          mt = u128_warp_sum(mt);
-          const U128 mw = u128_sub(u128_sub(mz, mh), mt);
-          wh = warp_sum_d(wh);
-          wt = warp_sum_d(wt);
-          nh = __reduce_add_sync(0xffffffffu, nh);
-          nw = __reduce_add_sync(0xffffffffu, nw);
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
-          if (row_ok && lane == 0) {
-            RangeRec rec;
-            rec.mh = mh;
-            rec.mt = mt;
-            rec.mw = mw;
-            rec.wh = wh;
-            rec.wt = wt;
-            rec.nh = nh;
-            rec.nw = nw;
-            rec.tmax = tmax;
-            rec.pad = 0u;
-            tb.rrec[row * p.nranges + g.range] = rec;
-          }
-        }
-        // the accumulator of the item: each warp its 32 dimensions of every row,
-        // the three parts added in fp64, fixed order
-        const int b = jj & 1;
-        const bool acc_ok = ok && mbar_wait(&accfull[b], (unsigned)(jj >> 1) & 1u) && !aborted(&s_abort);
-        if (bar_red_or(kGEpiBar, kGEpiThreads, !acc_ok)) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the brackets (and the logits) are complete
+    const float sc = p.scale2;
+    int t = 0, jj = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++jj) {
+      const GItem g = gitem_of(it, p);
+      const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
+      const int64_t row = (int64_t)g.group * p.gm + (int64_t)g.tile * RT + r;
+      const int nrows = min(RT, p.gm - g.tile * RT);
+      const bool row_ok = r < nrows;
+      float M = 0.0f;
+      int llo = INT_MIN, lhi = INT_MAX;
+      if (row_ok) {
+        const RowBracket bk = ld_cg_bracket(tb.brk + row);
+        M = bk.M;
+        llo = bk.llo;
+        lhi = bk.lhi;
+      }
+      U128 mz = u128_zero(), mh = u128_zero(), mt = u128_zero();
+      double wh = 0.0, wt = 0.0;  // fp64 sums of per-stage fp32 weight sums (for KL only)
+      uint32_t nh = 0u, nw = 0u;
+      float tmax = kNegInf;
+      unsigned long long* cand = tb.cand + row * kCandCap;
+      unsigned long long* cbuf = cbuf_all + wi * kCandBuf;
+      uint32_t nbuf = 0u;
+      for (int sg = s_lo; sg < s_hi && ok; ++sg, ++t) {
+        if (r >= RT || (t & 1) != h) continue;
+        const int slot = t % kGStages;
+        const int64_t k0 = (int64_t)sg * kGK + 4 * lane;  // this lane's four keys
+        // the stage's logits have landed; its slot's W tile is then free too
+        // (the MMAs that last read the slot have finished)
+        if (!mbar_wait(&ufull[h][slot], (unsigned)(t / (2 * kGStages)) & 1u) || aborted(&s_abort))
           ok = false;
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          if (lane == 0) s_abort = 1;  // the other warps stop waiting too
           break;
         }
-        tc_fence_after();
-        __syncwarp();
-        uint32_t c[32];
-        tc_ld32(lane_addr + (uint32_t)(b * kGN), c);
-        tc_fence_before();
-        mbar_arrive(&accempty[b]);
-        const int64_t row0 = (int64_t)g.group * p.gm + (int64_t)g.tile * RT;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row_ok) x = reinterpret_cast<const float4*>(uring + (slot * 4 + r) * kGK)[lane];
+        uint32_t hp[4][3], tp[4][3];
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        uint32_t winmask = 0u, hbits = 0u;
+        float sh_ = 0.0f, st_ = 0.0f;
+        // branch-free: every key is kept (level >= lhi), dropped (< llo) or window
 #pragma unroll
-        for (int rr = 0; rr < RT; ++rr) {
-          if (rr < nrows) {
+        for (int i = 0; i < 4; ++i) {
+          const bool valid = row_ok && k0 + i < p.n;
+          const float w = valid ? weight(xs[i], M, sc) : 0.0f;
+          const int L = key_level(xs[i], sc);
+          const bool head = valid && L >= lhi;
+          const bool tail = valid && L < llo;
+          const unsigned long long W = mass62(w);
+          u128_add(mz, W);
+          u128_add(mh, head ? W : 0ull);
+          u128_add(mt, tail ? W : 0ull);
+          nh += head ? 1u : 0u;
+          hbits |= head ? (1u << i) : 0u;
+          nw += (valid && !head && !tail) ? 1u : 0u;
+          winmask |= (valid && !head && !tail) ? (1u << i) : 0u;
+          sh_ += head ? w : 0.0f;
+          st_ += tail ? w : 0.0f;
+          tmax = fmaxf(tmax, tail ? xs[i] : kNegInf);
+          uint32_t pt[3];
+          split3(w, pt);
 #pragma unroll
-            for (int a = 0; a < (ERR ? 2 : 1); ++a) {
-              const double v = ((double)__uint_as_float(c[wcol<RT>(a, 0, rr)]) +
-                                (double)__uint_as_float(c[wcol<RT>(a, 1, rr)])) +
-                               (double)__uint_as_float(c[wcol<RT>(a, 2, rr)]);
-              acc_out[(((row0 + rr) * p.nranges + g.range) * 2 + a) * kGD + dim] = (float)v;
-            }
+          for (int part = 0; part < 3; ++part) {
+            hp[i][part] = head ? pt[part] : 0u;
+            if constexpr (ERR) tp[i][part] = tail ? pt[part] : 0u;
           }
         }
+        wh += (double)sh_;
+        wt += (double)st_;
+        // the stage's kept-for-certain bits: lane l holds keys 4 l .. 4 l + 3,
+        // i.e. bits 4 (l % 8) .. of word l / 8; eight lanes OR their nibbles
+        {
+          uint32_t wv = hbits << (4 * (lane & 7));
+          wv |= __shfl_xor_sync(0xffffffffu, wv, 1);
+          wv |= __shfl_xor_sync(0xffffffffu, wv, 2);
+          wv |= __shfl_xor_sync(0xffffffffu, wv, 4);
+          if (row_ok && (lane & 7) == 0) tb.hmask[row * tb.mask_words + 4 * (int64_t)sg + (lane >> 3)] = wv;
+        }
+        unsigned char* wtile = wring + slot * kGW;
+        const int c = lane >> 1;  // 16-byte piece (8 keys) along K; this lane writes one half
+        const uint32_t half = (uint32_t)(lane & 1) * 8u;
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(0, part, r), c, kGN) + half) =
+              make_uint2(hp[0][part] | (hp[1][part] << 16), hp[2][part] | (hp[3][part] << 16));
+          if constexpr (ERR)
+            *reinterpret_cast<uint2*>(wtile + sw128_offset(wcol<RT>(1, part, r), c, kGN) + half) =
+                make_uint2(tp[0][part] | (tp[1][part] << 16), tp[2][part] | (tp[3][part] << 16));
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wfull[slot]);
+        // window keys to this warp's buffer (flushed to the row's list when
+        // full and at the end of the item: one global atomic per flush)
+        if (__any_sync(0xffffffffu, winmask != 0u)) {
+          const uint32_t cnt = __popc(winmask);
+          uint32_t pre = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += y;
+          }
+          const uint32_t total = __shfl_sync(0xffffffffu, pre, 31);
+          if (nbuf + total > (uint32_t)kCandBuf) {
+            flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
+            nbuf = 0u;
+          }
+          uint32_t at = nbuf + pre - cnt;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (winmask & (1u << i)) cbuf[at++] = composite(order_key(xs[i]), (uint32_t)(k0 + i));
+          }
+          __syncwarp();
+          nbuf += total;  // a stage adds at most 128 <= kCandBuf keys
+        }
       }
-      if (!ok && lane == 0) {
-        atomicOr(status, CTA_DEV_TIMEOUT);
-        s_abort = 1;
+      if (row_ok && __any_sync(0xffffffffu, nbuf > 0u)) {
+        flush_cands(cbuf, nbuf, cand, tb.cand_cnt + row);
+        nbuf = 0u;
       }
+      // this warp's part of the range record (its stages); the warps of
+      // parity 1 hand theirs over in shared memory
+      const int b = jj & 1;
+      mz = u128_warp_sum(mz);
+      mh = u128_warp_sum(mh);
+      mt = u128_warp_sum(mt);
+      wh = warp_sum_d(wh);
+      wt = warp_sum_d(wt);
+      nh = __reduce_add_sync(0xffffffffu, nh);
+      nw = __reduce_add_sync(0xffffffffu, nw);
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+      if (h == 1 && lane == 0) rpart[b][r] = RecPart{mz, mh, mt, wh, wt, nh, nw, tmax};
+      // the accumulator of the item (all stages' MMAs done)
+      const bool acc_ok = ok && mbar_wait(&accfull[b], (unsigned)(jj >> 1) & 1u) && !aborted(&s_abort);
+      if (bar_red_or(kGEpiBar, kGEpiThreads, !acc_ok)) {
+        ok = false;
+        break;
+      }
+      if (h == 0 && row_ok && lane == 0) {
+        const RecPart& o = rpart[b][r];
+        u128_add(mz, o.mz);
+        u128_add(mh, o.mh);
+        u128_add(mt, o.mt);
+        RangeRec rec;
+        rec.mh = mh;
+        rec.mt = mt;
+        rec.mw = u128_sub(u128_sub(mz, mh), mt);
+        rec.wh = wh + o.wh;
+        rec.wt = wt + o.wt;
+        rec.nh = nh + o.nh;
+        rec.nw = nw + o.nw;
+        rec.tmax = fmaxf(tmax, o.tmax);
+        rec.pad = 0u;
+        tb.rrec[row * p.nranges + g.range] = rec;
+      }
+      tc_fence_after();
+      __syncwarp();
+      uint32_t c[32];
+      tc_ld32(lane_addr + (uint32_t)(b * kGN), c);
+      tc_fence_before();
+      mbar_arrive(&accempty[b]);
+      // each warp of the lane quarter writes every other (row, kept/dropped) sum,
+      // the three parts added in fp64, fixed order
+      const int64_t row0 = (int64_t)g.group * p.gm + (int64_t)g.tile * RT;
+      constexpr int NA = ERR ? 2 : 1;
+#pragma unroll
+      for (int x = 0; x < RT * NA; ++x) {
+        const int rr = x / NA, a = x % NA;
+        if ((x & 1) == h && rr < nrows) {
+          const double v = ((double)__uint_as_float(c[wcol<RT>(a, 0, rr)]) +
+                            (double)__uint_as_float(c[wcol<RT>(a, 1, rr)])) +
+                           (double)__uint_as_float(c[wcol<RT>(a, 2, rr)]);
+          acc_out[(((row0 + rr) * p.nranges + g.range) * 2 + a) * kGD + dim] = (float)v;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      atomicOr(status, CTA_DEV_TIMEOUT);
+      s_abort = 1;
     }
   }
 
@@ -787,7 +842,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
 }
 
 template <int RT, bool ERR>
-cudaError_t launch_t(const CUtensorMap& map, const float* u, const float* cmax, const TcBufs& tb,
+cudaError_t launch_t(const CUtensorMap& map, const float* u, const unsigned char* vbase, const TcBufs& tb,
                      float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   auto kern = gather_tc_kernel<RT, ERR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
@@ -805,16 +860,16 @@ cudaError_t launch_t(const CUtensorMap& map, const float* u, const float* cmax, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, u, cmax, tb, acc, p, status);
+  return cudaLaunchKernelEx(&cfg, kern, map, u, vbase, tb, acc, p, status);
 }
 
 template <bool ERR>
-cudaError_t launch_e(const CUtensorMap& map, const float* u, const float* cmax, const TcBufs& tb,
+cudaError_t launch_e(const CUtensorMap& map, const float* u, const unsigned char* vbase, const TcBufs& tb,
                      float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   switch (p.rt_out) {
-    case 1: return launch_t<1, ERR>(map, u, cmax, tb, acc, p, status, st);
-    case 2: return launch_t<2, ERR>(map, u, cmax, tb, acc, p, status, st);
-    case 4: return launch_t<4, ERR>(map, u, cmax, tb, acc, p, status, st);
+    case 1: return launch_t<1, ERR>(map, u, vbase, tb, acc, p, status, st);
+    case 2: return launch_t<2, ERR>(map, u, vbase, tb, acc, p, status, st);
+    case 4: return launch_t<4, ERR>(map, u, vbase, tb, acc, p, status, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -864,9 +919,9 @@ void set_ranges_tc(Plan* p, int sms) {
   const int64_t spu = (p->n + kGK - 1) / kGK;
   // range partials fit the workspace (one slot per chunk); at most 1024 ranges are tried
   const int64_t cap = std::min<int64_t>(std::min<int64_t>(spu, p->nchunks), 1024);
-  // A work item starts with the row bracket (a few microseconds: about ten
-  // stages of streaming), so the planner charges that much per item.
-  constexpr int64_t kItemCost = 10;
+  // A work item ends with the accumulator hand-over and the range record
+  // (about two stages of streaming), so the planner charges that much per item.
+  constexpr int64_t kItemCost = 2;
   // Every range count is scored by the busiest CTA's items times their length
   // (items go round-robin over the grid); the eight best are then simulated
   // exactly (the last range of a unit is shorter).
@@ -924,8 +979,24 @@ cudaError_t launch_gather_tc(const void* V, const float* u, const float* cmax, c
   if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
   if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
-  return p.want_err ? launch_e<true>(map, u, cmax, tb, acc, p, status, st)
-                    : launch_e<false>(map, u, cmax, tb, acc, p, status, st);
+  // the row brackets, then the value pass (both programmatic dependents)
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.rows, 1, 1);
+    cfg.blockDim = dim3(kBThreads, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, bracket_tc_kernel, (const RangeHist*)tb.hist,
+                                             cmax, tb.brk, p);
+    if (e != cudaSuccess) return e;
+  }
+  const unsigned char* vb = static_cast<const unsigned char*>(V);
+  return p.want_err ? launch_e<true>(map, u, vb, tb, acc, p, status, st)
+                    : launch_e<false>(map, u, vb, tb, acc, p, status, st);
 }
 
 }  // namespace cta

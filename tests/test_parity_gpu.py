@@ -162,6 +162,64 @@ def test_back_to_back_calls_share_one_workspace(want_err):
             compare(sub, 0.01, g, o, rows=group_rows(prob, 0, kvh))
 
 
+@pytest.mark.parametrize("last_write", ["K", "V", "q"])
+def test_inputs_written_by_the_preceding_kernel(last_write):
+    # The caller appends the new key and value rows and writes the query with
+    # its own kernels on the same stream, immediately before each call, with
+    # no host synchronisation.  The new key is made to dominate the query's
+    # logits, so a pass that read K, V or q before those kernels finished
+    # would select or weight the wrong rows.  `last_write` is the tensor the
+    # kernel just before the call writes.
+    prob = W.decode128k(batch=1, n=40000, steps=4)
+    dev = torch.device("cuda")
+    g = prob.n_heads // prob.n_kv_heads
+    K, V = prob.K.to(dev), prob.V.to(dev)
+    q_dev = torch.zeros_like(prob.q, device=dev)
+    ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                            batch=prob.batch), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    rng = np.random.default_rng(77)
+    steps = []
+    for t in range(4):
+        q_t = prob.meta["q_steps"][t]                          # [1, heads, 1, d]
+        # a key along the summed queries of each KV group, scaled up
+        qsum = q_t.float().reshape(prob.n_kv_heads, g, prob.d).sum(1)
+        k_new = (qsum / qsum.norm(dim=1, keepdim=True) * (3.0 + t)).to(torch.bfloat16)
+        v_new = torch.from_numpy(rng.standard_normal((prob.n_kv_heads, prob.d)).astype(np.float32) * 4.0
+                                 ).to(torch.bfloat16)
+        steps.append((q_t, k_new, v_new))
+    writes_dev = [(a.to(dev), b.to(dev), c.to(dev)) for a, b, c in steps]
+    torch.cuda.synchronize()
+    big = torch.zeros(64 << 20, dtype=torch.float32, device=dev)  # delays the stream a little
+    results = []
+    for t, (q_t, k_new, v_new) in enumerate(writes_dev):
+        big.add_(1.0)
+        writes = {"q": lambda: q_dev.copy_(q_t),
+                  "K": lambda: K[0, :, -1, :].copy_(k_new),
+                  "V": lambda: V[0, :, -1, :].copy_(v_new)}
+        for name in [x for x in ("q", "K", "V") if x != last_write] + [last_write]:
+            writes[name]()
+        results.append(cta.cta_certified_topk_attn(q_dev, K, V, 0.01, workspace=ws,
+                                                   status_dev=status, want_err=True,
+                                                   want_kl=True, want_gap=True))
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    K_h, V_h = prob.K.clone(), prob.V.clone()
+    for t, (q_t, k_new, v_new) in enumerate(steps):
+        K_h[0, :, -1, :] = k_new
+        V_h[0, :, -1, :] = v_new
+        mod = W.Problem(prob.name, q_t.clone(), K_h.clone(), V_h.clone(), prob.eps, prob.batch,
+                        prob.n_heads, prob.n_kv_heads, prob.m, prob.n, prob.d)
+        gres = to_host(results[t])
+        for kvh in (0, 3, 7):
+            sub = sub_problem(mod, 0, kvh)
+            o = run_oracle(sub, 0.01)
+            rows = group_rows(prob, 0, kvh)
+            # the new key is among the kept keys of every row of the group
+            assert all(prob.n - 1 in o["idx"][j] for j in range(len(rows)))
+            compare(sub, 0.01, gres, o, rows=rows)
+
+
 def test_bert_small_all_query():
     prob = W.bert(batch=1, n_heads=4, n=512, d=64, sharp_from=2)
     g, o, rep = check(prob, prob.eps, "bert small")
