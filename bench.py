@@ -3,9 +3,14 @@
 Headline workload: 128K GQA decode - batch 1, 32 query heads, 8 KV heads,
 d = 128, n = 131072 bf16 KV cache with sink / recent-window / needle
 structure, eps = 0.01, a fresh query set every step (64-step cycle).  One
-step = one call of cta_certified_topk_attn over all 32 query heads (logits,
-certified selection, head/tail value sums, finalisation, err and KL on).
-The metric is query heads per second; the roofline is HBM bandwidth.
+step = one call of cta_certified_topk_attn over all 32 query heads: four
+kernels (logits with level histograms, row brackets, the bracketed value
+pass, the exact cut with indices and outputs), err and KL on.  The metric is
+query heads per second; the roofline is HBM bandwidth.  Also reported: the
+same workload at eps = 0.1, the 32K decode (batch 4), end-to-end rates
+through the C ABI with host buffers (with and without the indices), the tiny
+config's microseconds per call, the Gaussian sweep and the BERT-shaped
+all-query workload.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libcta|reference]
 
@@ -33,8 +38,12 @@ sys.path.insert(0, ROOT)
 METRIC = "certified top-k attn query-heads/s & HBM GB/s (% of peak) at n=32K/128K"
 UNIT = "query-heads/s"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("score.cu", "score_kv_tc.cu", "select.cu", "gather.cu", "gather_tc.cu",
-                  "finalize.cuh", "umma.cuh", "common.cuh")
+KERNEL_SOURCES = ("score_kv_tc.cu", "gather_tc.cu", "settle_tc.cu", "umma.cuh", "common.cuh")
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the measured copy peak is the roofline's denominator)
+# the four kernels of one decode call (bf16 K, V with d = 128), in launch order
+DECODE_PHASES = ("logits", "brackets", "values", "settle")
+DECODE_KERNELS = {"logits": "score_kv_tc_kernel", "brackets": "bracket_tc_kernel",
+                  "values": "gather_tc_kernel", "settle": "settle_tc_kernel"}
 
 
 # --------------------------------------------------------------------------
@@ -165,13 +174,16 @@ class ClockSampler:
 def algorithmic_bytes(prob, k_rows=None) -> dict:
     """Bytes one step must move at minimum: K once per KV head for the logits,
     every V row once per KV head for the output (the exact head-tail error
-    needs the dropped rows too), q and outputs (negligible), and the kept
-    indices written (reported separately)."""
+    needs the dropped rows too; at k/n ~ 0.9 with four query heads per KV head
+    the union of the kept rows is every row as well), q and outputs
+    (negligible), and the kept indices written (reported separately).  Per
+    kernel: the logits pass reads K, the value pass reads V, the last kernel
+    writes the indices (and reads one bit per key of the kept-for-certain mask)."""
     kv = prob.batch * prob.n_kv_heads * prob.n * prob.d * prob.K.element_size()
     idx = 0 if k_rows is None else int(k_rows.sum()) * 4
-    logits = 4 * prob.rows * prob.n
-    # selection: read every row's fp32 logits once, write the kept indices
-    return {"score": kv, "select": logits + idx, "gather": kv, "step": 2 * kv, "idx_write": idx}
+    mask = prob.rows * prob.n // 8
+    return {"logits": kv, "brackets": 0, "values": kv, "settle": idx + mask, "step": 2 * kv,
+            "idx_write": idx}
 
 
 def run_libcta(args, rank, world, local_rank) -> dict | None:
@@ -337,10 +349,52 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     h2d = q_steps[0].numel() * q_steps[0].element_size()
     d2h = out.numel() * out.element_size() + 4 * rows * 4
 
+    # The same, with the kept indices copied back too (idx is the largest
+    # result: rows x n int32 per step; the copy crosses PCIe and bounds the rate).
+    ei_steps = max(1, min(args.steps, 200))
+    host_idx = [torch.empty_like(idx, device="cpu").pin_memory() for _ in range(2)]
+    dev_idx = [idx, torch.empty_like(idx)]
+
+    def e2e_idx_step(t):
+        b = t % 2
+        stream.wait_event(ev_ready[b])
+        sm = dev_small[b]
+        cta.cta_certified_topk_attn(dev_q[b], K, V, eps, out=dev_out[b],
+                                    k_out=sm[0].view(torch.int32), idx_out=dev_idx[b], tv_out=sm[1],
+                                    err_out=sm[2], kl_out=sm[3], workspace=ws, status_dev=status,
+                                    stream=stream)
+        ev_done[b].record(stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(ev_done[b])
+            host_out[b].copy_(dev_out[b], non_blocking=True)
+            host_small[b].copy_(sm, non_blocking=True)
+            host_idx[b].copy_(dev_idx[b], non_blocking=True)
+            dev_q[b].copy_(host_q[(t + 2) % nq], non_blocking=True)
+            ev_ready[b].record(copy)
+
+    torch.cuda.synchronize(device)
+    e2e_prime(0)
+    for t in range(3):
+        e2e_idx_step(t)
+    torch.cuda.synchronize(device)
+    barrier(dist, device)
+    s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s3.record(stream)
+    e2e_prime(0)
+    for t in range(ei_steps):
+        e2e_idx_step(t)
+    stream.wait_event(ev_ready[(ei_steps - 1) % 2])
+    e3.record(stream)
+    torch.cuda.synchronize(device)
+    ei_seconds = max_over_ranks(s3.elapsed_time(e3) / 1e3, dist, device)
+    last = (ei_steps - 1) % 2
+    assert torch.equal(host_idx[last], dev_idx[last].cpu()), "e2e indices differ from the device's"
+    d2h_idx = d2h + idx.numel() * idx.element_size()
+
     assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
     nbytes = algorithmic_bytes(prob, k_out.reshape(-1).cpu())
     peak, peak_kind = measured_peaks()
-    names = ("score", "select", "gather", "finalize")
+    names = DECODE_PHASES
     dom = max(range(4), key=lambda j: phase[j])
     dom_name = names[dom]
     dom_bytes = nbytes.get(dom_name, 0)
@@ -349,6 +403,11 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
     ne_dom = max(range(4), key=lambda j: ne_phase[j])
     ne_bytes = nbytes.get(names[ne_dom], 0)
     ne_achieved = ne_bytes / (ne_phase[ne_dom] / 1e3) / 1e9 if ne_bytes else None
+    kernel_rates = {
+        nm: {"kernel": DECODE_KERNELS[nm], "ms": round(phase[j], 5),
+             "algorithmic_bytes": nbytes[nm],
+             "gbs": (nbytes[nm] / (phase[j] / 1e3) / 1e9) if nbytes[nm] and phase[j] > 0 else None}
+        for j, nm in enumerate(names)}
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": seconds * 1e3 / args.steps,
@@ -364,14 +423,22 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
-            "bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak if achieved else None, "traffic": profiled_traffic(dom_name),
+            "bound": "hbm", "kernel": DECODE_KERNELS[dom_name], "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak if achieved else None,
+            "traffic": profiled_traffic(DECODE_KERNELS[dom_name]),
             "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_kind,
         },
         "step_roofline": {"achieved_gbs": step_gbs, "frac": step_gbs / peak,
+                          "peak": peak, "peak_source": peak_kind,
+                          "frac_of_nominal": step_gbs / NOMINAL_HBM_GBS,
+                          "nominal_peak": NOMINAL_HBM_GBS,
                           "algorithmic_bytes_per_step": nbytes["step"],
-                          "idx_write_bytes_per_step": nbytes["idx_write"]},
+                          "idx_write_bytes_per_step": nbytes["idx_write"],
+                          "note": "the whole step (K and V once, ms_per_step) against the measured "
+                                  "copy peak and the nominal 8 TB/s; 'roofline' is the dominant "
+                                  "kernel alone"},
         "phase_ms": dict(zip(names, [round(p, 5) for p in phase])),
+        "kernels": kernel_rates,
         "phase_region": {"ms_per_step": phased_seconds * 1e3 / args.steps,
                          "note": "phase_ms and the roofline come from a second run of the same "
                                  "steps with CUDA events between the kernels (which serialise "
@@ -383,19 +450,24 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
                         "neighbouring steps' kernels (double-buffered, one event wait per step "
                         "on the compute stream); the KV cache is resident and idx stays on "
                         "the device"},
+        "e2e_with_idx": {"value": aggregate(rows, ei_steps, world, ei_seconds), "unit": UNIT,
+                         "steps": ei_steps, "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": d2h_idx,
+                         "note": "as e2e, with idx_out ([rows, n] int32) also copied back to pinned "
+                                 "host memory every step; 'e2e' (idx left on the device, as a "
+                                 "decode loop keeps it) is the headline"},
         "no_err": {
             "value": aggregate(rows, ne_steps, world, ne_seconds), "unit": UNIT,
             "steps": ne_steps, "ms_per_step": ne_seconds * 1e3 / ne_steps,
             "phase_ms": dict(zip(names, [round(p, 5) for p in ne_phase])),
-            "roofline": {"bound": "hbm", "kernel": names[ne_dom], "achieved": ne_achieved,
+            "roofline": {"bound": "hbm", "kernel": DECODE_KERNELS[names[ne_dom]], "achieved": ne_achieved,
                          "peak": peak, "unit": "GB/s",
                          "frac": ne_achieved / peak if ne_achieved else None,
                          "algorithmic_bytes_per_launch": ne_bytes},
             "note": "err_out and kl_out not requested; timed after the main region",
         },
-        # logits, selection, value sums, and (bf16 values with d = 128: the
-        # tensor-core value pass) a separate row-parallel finalisation kernel
-        "gpu_launches": (4 if (prob.V.dtype == torch.bfloat16 and prob.d == 128) else 3) * args.steps,
+        # logits, row brackets, value pass, cut/indices/outputs: four per call
+        "gpu_launches": 4 * args.steps,
         "k_over_n_mean": float(k_out.float().mean().item() / prob.n),
         "clocks": clocks.summary(),
     }
@@ -485,6 +557,104 @@ def run_all_query(steps: int, warmup: int) -> dict:
                         "steps": steps, "warmup": warmup, "k_over_n_mean":
                             float(k_out.float().mean().item() / prob.n)}
     return result
+
+
+def run_tiny(steps: int, warmup: int) -> dict:
+    """The tiny Gaussian-score workload (batch 1, 8 heads, d = 64, n = 1024,
+    fp32, eps = 0.01): microseconds per call, back to back on one stream
+    (launch-bound: three kernels per call)."""
+    import torch
+    import certified_top_sparse_b200 as cta
+    from certified_top_sparse_b200 import workloads as W
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    prob = W.tiny()
+    q, K, V = prob.q.to(device), prob.K.to(device), prob.V.to(device)
+    rshape = (prob.batch, prob.n_heads, prob.m)
+    out = torch.empty_like(q)
+    k_out = torch.empty(rshape, dtype=torch.int32, device=device)
+    idx = torch.empty((*rshape, prob.n), dtype=torch.int32, device=device)
+    tv = torch.empty(rshape, dtype=torch.float32, device=device)
+    err = torch.empty(rshape, dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                            batch=prob.batch, dtype=cta.CTA_F32),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        cta.cta_certified_topk_attn(q, K, V, prob.eps, out=out, k_out=k_out, idx_out=idx,
+                                    tv_out=tv, err_out=err, workspace=ws, status_dev=status,
+                                    stream=stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
+    us = a.elapsed_time(b) / steps * 1e3
+    return {"us_per_call": us, "unit": "us/call", "steps": steps, "gpu_launches_per_call": 3,
+            "config": {"workload": "tiny: batch 1, 8 heads, d=64, n=1024, fp32, Gaussian scores "
+                                   "(sigma 1, 2, 3 over the heads), eps=0.01, err on"},
+            "k_over_n_mean": float(k_out.float().mean().item() / prob.n)}
+
+
+def run_sweep(reps: int) -> dict:
+    """The Gaussian-score sweep (fp32, d = 64, 256 query rows sharing one K per
+    cell): per (n, sigma, eps) cell the time per call (the mean of `reps`
+    calls), the logits' FMA rate and the mean k/n beside the Gaussian rule
+    Phi_c(sigma + Phi^-1(eps))."""
+    import torch
+    import certified_top_sparse_b200 as cta
+    from certified_top_sparse_b200 import workloads as W
+    from statistics import NormalDist
+
+    device = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(device)
+    nd = NormalDist()
+    cells = []
+    for n in W.SWEEP_N:
+        for sigma in W.SWEEP_SIGMA:
+            prob = W.sweep_cell(n, sigma)
+            q, K, V = prob.q.to(device), prob.K.to(device), prob.V.to(device)
+            rshape = (prob.batch, prob.n_heads, prob.m)
+            out = torch.empty_like(q)
+            k_out = torch.empty(rshape, dtype=torch.int32, device=device)
+            idx = torch.empty((*rshape, prob.n), dtype=torch.int32, device=device)
+            tv = torch.empty(rshape, dtype=torch.float32, device=device)
+            status = torch.zeros(1, dtype=torch.int32, device=device)
+            ws = torch.empty(cta.cta_workspace_size(prob.n, prob.d, prob.n_heads, prob.n_kv_heads,
+                                                    m=prob.m, dtype=cta.CTA_F32),
+                             dtype=torch.uint8, device=device)
+            for eps in W.SWEEP_EPS:
+                def step():
+                    cta.cta_certified_topk_attn(q, K, V, eps, out=out, k_out=k_out, idx_out=idx,
+                                                tv_out=tv, workspace=ws, status_dev=status,
+                                                stream=stream)
+                for _ in range(2):
+                    step()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                for _ in range(reps):
+                    step()
+                b.record(stream)
+                torch.cuda.synchronize(device)
+                assert int(status.item()) == 0, f"device status {int(status.item()):#x}"
+                us = a.elapsed_time(b) / reps * 1e3
+                rule = 1.0 - nd.cdf(sigma + nd.inv_cdf(eps))
+                cells.append({"n": n, "sigma": sigma, "eps": eps, "us_per_call": round(us, 2),
+                              "logit_tflops": 2.0 * prob.m * n * prob.d / (us * 1e-6) / 1e12,
+                              "k_over_n": float(k_out.float().mean().item() / n),
+                              "gaussian_rule": rule})
+            del q, K, V, idx, ws
+    return {"cells": cells, "unit": "us/call",
+            "config": {"workload": "Gaussian-score sweep: fp32, d=64, 256 query rows per cell "
+                                   "sharing K ~ N(0, I), |q| = sigma sqrt(d); n x sigma x eps = "
+                                   "4 x 4 x 3 cells", "reps_per_cell": reps}}
 
 
 # --------------------------------------------------------------------------
@@ -578,6 +748,8 @@ def main(argv=None):
                     help="also measure this workload (same method, fewer steps) and nest it")
     ap.add_argument("--all-query", choices=("bert", "none"), default="bert",
                     help="also measure the BERT-shaped all-query workload (tensor-core path)")
+    ap.add_argument("--no-extras", dest="extras", action="store_false",
+                    help="skip the eps = 0.1 line, the tiny-call timing and the Gaussian sweep")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -594,6 +766,16 @@ def main(argv=None):
             res["secondary"] = {k: r2[k] for k in ("value", "ms_per_step", "config", "roofline",
                                                    "step_roofline", "phase_ms", "k_over_n_mean",
                                                    "no_err")}
+        if res is not None and world == 1 and args.extras and args.workload == "decode128k":
+            # the same workload at eps = 0.1 (the other eps the 128K config names)
+            sub = argparse.Namespace(**{**vars(args), "eps": 0.1, "steps": max(100, args.steps // 2)})
+            r3 = run_libcta(sub, rank, world, local_rank)
+            res["eps_0.1"] = {k: r3[k] for k in ("value", "ms_per_step", "config", "roofline",
+                                                 "step_roofline", "phase_ms", "k_over_n_mean",
+                                                 "e2e")}
+        if res is not None and world == 1 and args.extras:
+            res["tiny"] = run_tiny(steps=max(200, args.steps // 2), warmup=args.warmup)
+            res["sweep"] = run_sweep(reps=5)
         if res is not None and args.all_query != "none" and world == 1:
             res["all_query"] = run_all_query(steps=max(20, args.steps // 40), warmup=args.warmup)
         if res is not None and world == 1 and not args.no_cpu_baseline:

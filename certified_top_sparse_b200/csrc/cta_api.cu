@@ -239,8 +239,9 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
 
   if (record(ev, 0, st) != CTA_OK) return CTA_ERR_CUDA;
   if (gtc) {
-    // tensor-core decode path: logits (+ level histograms), the bracketed
-    // value pass (+ exact masses), then the exact cut, indices and outputs
+    // tensor-core decode path: logits (+ level histograms), the row brackets,
+    // the bracketed value pass (+ exact masses), then the exact cut, indices
+    // and outputs; the events fall between the four kernels
     TcBufs tb;
     tb.hist = reinterpret_cast<RangeHist*>(ws + L.hist);
     tb.rrec = reinterpret_cast<RangeRec*>(ws + L.rrec);
@@ -253,12 +254,13 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
     tb.mask_words = mask_words(p);
     if (launch_score_kv_tc(q, K, u, cmax, tb, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
     if (record(ev, 1, st) != CTA_OK) return CTA_ERR_CUDA;
-    if (launch_gather_tc(V, u, cmax, tb, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+    if (launch_bracket_tc(cmax, tb, p, st) != cudaSuccess) return CTA_ERR_CUDA;
     if (record(ev, 2, st) != CTA_OK) return CTA_ERR_CUDA;
+    if (launch_gather_tc(V, u, tb, acc, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;
+    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
     if (launch_settle_tc(V, u, tb, acc, out, k_out, idx_out, tv_out, opts->err_out, opts->kl_out,
                          opts->gap_out, p, status, st) != cudaSuccess)
       return CTA_ERR_CUDA;
-    if (record(ev, 3, st) != CTA_OK) return CTA_ERR_CUDA;
     if (record(ev, 4, st) != CTA_OK) return CTA_ERR_CUDA;
     return CTA_OK;
   }

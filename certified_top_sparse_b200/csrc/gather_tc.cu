@@ -974,26 +974,24 @@ void set_ranges_tc(Plan* p, int sms) {
   p->nranges = (int)best_nr;
 }
 
-cudaError_t launch_gather_tc(const void* V, const float* u, const float* cmax, const TcBufs& tb,
-                             float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
+cudaError_t launch_bracket_tc(const float* cmax, const TcBufs& tb, const Plan& p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.rows, 1, 1);
+  cfg.blockDim = dim3(kBThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, bracket_tc_kernel, (const RangeHist*)tb.hist, cmax, tb.brk, p);
+}
+
+cudaError_t launch_gather_tc(const void* V, const float* u, const TcBufs& tb, float* acc,
+                             const Plan& p, uint32_t* status, cudaStream_t st) {
   if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
   if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
-  // the row brackets, then the value pass (both programmatic dependents)
-  {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.rows, 1, 1);
-    cfg.blockDim = dim3(kBThreads, 1, 1);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, bracket_tc_kernel, (const RangeHist*)tb.hist,
-                                             cmax, tb.brk, p);
-    if (e != cudaSuccess) return e;
-  }
   const unsigned char* vb = static_cast<const unsigned char*>(V);
   return p.want_err ? launch_e<true>(map, u, vb, tb, acc, p, status, st)
                     : launch_e<false>(map, u, vb, tb, acc, p, status, st);

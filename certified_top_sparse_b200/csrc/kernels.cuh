@@ -53,14 +53,15 @@ cudaError_t launch_select_short(const float* u, RowSel* sel, int32_t* k_out, flo
 // dropped) keys, then (the last CTA of each (KV group, row tile), counted in
 // unit_cnt, which selection zeroes) out, err, KL and the single-gap bound.
 // gather_ctas_per_sm: the CTAs per SM its launch is planned for.
-// The tensor-core decode path (bf16 q, K, V with d = 128), three kernels:
+// The tensor-core decode path (bf16 q, K, V with d = 128), four kernels:
 //   launch_score_kv_tc: logits (TMA-fed K stages, the row tile's queries as the
 //     B operand), one partial maximum per row and range (Plan::nmax) and the
 //     per-range level histograms; zeroes tb.cand_cnt and tb.ticket;
-//   launch_gather_tc: the value pass after set_ranges_tc: brackets every row's
-//     cut from the histograms, value sums of the keys on either side of the
-//     bracket (range partials in acc), exact masses (tb.rrec), window
-//     candidates (tb.cand) and the brackets (tb.brk);
+//   launch_bracket_tc: every row's bracket of the cut (tb.brk) from the
+//     histograms and maxima, one CTA per row;
+//   launch_gather_tc: the value pass after set_ranges_tc: value sums of the
+//     keys on either side of the bracket (range partials in acc), exact masses
+//     (tb.rrec), window candidates (tb.cand) and the kept-for-certain mask;
 //   launch_settle_tc: the exact cut, the kept indices and the outputs.
 bool gather_tc_applies(const Plan& p, int dtype);
 cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cmax,
@@ -70,8 +71,9 @@ cudaError_t launch_score_kv_tc(const void* q, const void* K, float* u, float* cm
 // of 64 dimensions x 128 keys (the stages of the streaming tensor-core kernels).
 bool encode_kv_map(CUtensorMap* map, const void* base, const Plan& p);
 void set_ranges_tc(Plan* p, int sms);
-cudaError_t launch_gather_tc(const void* V, const float* u, const float* cmax, const TcBufs& tb,
-                             float* acc, const Plan& p, uint32_t* status, cudaStream_t st);
+cudaError_t launch_bracket_tc(const float* cmax, const TcBufs& tb, const Plan& p, cudaStream_t st);
+cudaError_t launch_gather_tc(const void* V, const float* u, const TcBufs& tb, float* acc,
+                             const Plan& p, uint32_t* status, cudaStream_t st);
 cudaError_t launch_settle_tc(const void* V, const float* u, const TcBufs& tb, float* acc, void* out,
                              int32_t* k_out, int32_t* idx_out, float* tv_out, float* err_out,
                              float* kl_out, float* gap_out, const Plan& p, uint32_t* status,

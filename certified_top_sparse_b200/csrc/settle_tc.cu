@@ -62,10 +62,13 @@ constexpr int kSubMax = 512;             // sub-level bins of the cut search
 constexpr int kSubList = 256;            // keys of the cut's sub-level that are sorted
 constexpr int kWList = 256;              // per-warp list of window keys awaiting their value rows
 constexpr int kMaskBlock = 4 * kTThreads;  // mask words per block of the index writes (4 per thread)
-constexpr int kVPre = 64;                // window value rows copied in while the cut is searched
+constexpr int kVPre = 128;
+constexpr int kStageWords = 124;         // mask words per staging round (124 x 32 + 3 <= 4096 slots)               // window value rows copied in while the cut is searched
+
+static_assert(kCandCap * 2 >= kStageWords * 32 + 3, "the candidate list doubles as the staging area");
 
 struct SettleShared {
-  unsigned long long cand[kCandCap];     // the row's candidates (sorted in place by the fallback)
+  alignas(16) unsigned long long cand[kCandCap];  // the row's candidates (sorted in place by the fallback)
   union {
     struct {
       unsigned long long lo[kSubMax], hi[kSubMax];  // exact sub-level masses, 128-bit
@@ -83,8 +86,9 @@ struct SettleShared {
       uint32_t off[kMaskBlock];   // exclusive offsets of the words' kept keys
     } mk;
   } u;
-  uint32_t mask0[kMaskBlock];            // the segment's first block of kept-for-certain words
-  uint2 vrow[kVPre][kTD / 4];            // value rows of the segment's first window keys
+  alignas(16) uint32_t mask0[kMaskBlock];  // the segment's first block of kept-for-certain words
+  alignas(16) uint2 vrow[kVPre][kTD / 4];  // value rows of the segment's first window keys
+  unsigned long long bar_in, bar_v;        // bulk copies: candidates and mask words; value rows
   unsigned long long wl_key[kTWarps][kWList];  // window key: logit bits (high 32) | index (low 32)
   unsigned char wl_kept[kTWarps][kWList];
   float accw[2][kTWarps][kTD];           // per-warp window value sums (kept, dropped)
@@ -101,18 +105,18 @@ struct SettleShared {
   int found, jstar, last;
 };
 
-// 16-byte asynchronous copy global -> shared (L2 only), and its group waits.
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+// Bulk copy shared -> global (async proxy), its commit and waits.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ U128 u128_make(unsigned long long lo, unsigned long long hi) {
   return U128{lo, hi};
@@ -124,7 +128,7 @@ __device__ __forceinline__ double warp_sum_dbl(double v) {
 }
 
 // Exclusive scan of one 128-bit and one 32-bit value per thread over the block.
-__device__ void block_excl_scan(U128& v, uint32_t& c, SettleShared& S) {
+__device__ __noinline__ void block_excl_scan(U128& v, uint32_t& c, SettleShared& S) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   U128 x = v;
   uint32_t y = c;
@@ -158,7 +162,7 @@ __device__ void block_excl_scan(U128& v, uint32_t& c, SettleShared& S) {
 
 // Exclusive scan of two packed 64-bit words per thread (four 16-bit counts
 // each, no field overflows); tot gets the block totals.
-__device__ void block_excl_scan_packed(unsigned long long* v, unsigned long long* tot,
+__device__ __noinline__ void block_excl_scan_packed(unsigned long long* v, unsigned long long* tot,
                                        SettleShared& S) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned long long x0 = v[0], x1 = v[1];
@@ -228,6 +232,292 @@ __device__ __forceinline__ float ck_logit(unsigned long long ck) {
   return key_value((uint32_t)(ck >> 32));
 }
 
+// Cold path of the cut search: the whole candidate list sorted (bitonic) and
+// walked from the top.  Sets S.cut, S.C, S.k and S.found; returns S.found.
+__device__ __noinline__ bool cut_by_sort(SettleShared& S, int m, float M, float sc, uint32_t NH,
+                                         U128 Z, U128 base, double eps) {
+  const int tid = threadIdx.x;
+  // the whole candidate list sorted, then walked from the top
+  int P = 1;
+  while (P < m) P <<= 1;
+  for (int i = m + tid; i < P; i += kTThreads) S.cand[i] = 0ull;  // pad below all keys
+  __syncthreads();
+  bitonic_sort_desc(S.cand, P);
+  constexpr int E = kCandCap / kTThreads;
+  unsigned long long Wl[E];
+  U128 ls = u128_zero();
+#pragma unroll
+  for (int j = 0; j < E; ++j) {
+    const int i = tid * E + j;
+    Wl[j] = (i < m) ? mass62(weight(ck_logit(S.cand[i]), M, sc)) : 0ull;
+    u128_add(ls, Wl[j]);
+  }
+  U128 cum = ls;
+  uint32_t dummy = 0u;
+  block_excl_scan(cum, dummy, S);
+  u128_add(cum, base);
+  U128 end = cum;
+  u128_add(end, ls);
+  if (!certified128(Z, cum, eps) && certified128(Z, end, eps)) {
+#pragma unroll
+    for (int j = 0; j < E; ++j) {
+      const int i = tid * E + j;
+      U128 nx = cum;
+      u128_add(nx, Wl[j]);
+      if (i < m && certified128(Z, nx, eps)) {
+        S.C = nx;
+        S.cut = S.cand[i];
+        S.k = (long long)NH + i + 1;
+        S.found = 1;
+        break;
+      }
+      cum = nx;
+    }
+  }
+  __syncthreads();
+  return S.found != 0;
+}
+
+// Cold path of the cut search (candidate list overflowed or the bracket was
+// rejected): radix select over the composite keys of the window's logits,
+// eight bits per pass.  Sets S.cut, S.C and S.k.
+__device__ __noinline__ void cut_by_radix(SettleShared& S, const float* __restrict__ ur, int64_t n,
+                                          float M, float sc, int llo, int lhi, uint32_t NH, U128 Z,
+                                          U128 base, double eps, uint32_t* __restrict__ status) {
+  const int tid = threadIdx.x;
+  // radix select over the window's composite keys, eight bits per pass
+  unsigned long long prefix = 0ull;
+  U128 bs = base;
+  uint32_t above = 0u;
+  bool ok = true;
+  for (int level = 0; level < 8 && ok; ++level) {
+    const int shift = 56 - 8 * level;
+    for (int i = tid; i < 256; i += kTThreads) {
+      S.u.rx.lo[i] = 0ull;
+      S.u.rx.hi[i] = 0ull;
+      S.u.rx.cnt[i] = 0u;
+    }
+    __syncthreads();
+    for (int64_t key = tid; key < n; key += kTThreads) {
+      const float x = __ldcg(ur + key);
+      if (!in_window(x, sc, llo, lhi)) continue;
+      const unsigned long long ck = composite(order_key(x), (uint32_t)key);
+      if (level > 0 && (ck >> (64 - 8 * level)) != prefix) continue;
+      const int dig = (int)((ck >> shift) & 0xffull);
+      const unsigned long long w = mass62(weight(x, M, sc));
+      const unsigned long long old = atomicAdd(&S.u.rx.lo[dig], w);
+      if (old + w < old) atomicAdd(&S.u.rx.hi[dig], 1ull);
+      atomicAdd(&S.u.rx.cnt[dig], 1u);
+    }
+    __syncthreads();
+    // digits in descending order: thread t < 256 owns digit 255 - t
+    U128 dm = u128_zero();
+    uint32_t dc = 0u;
+    if (tid < 256) {
+      dm = u128_make(S.u.rx.lo[255 - tid], S.u.rx.hi[255 - tid]);
+      dc = S.u.rx.cnt[255 - tid];
+    }
+    U128 mex = dm;
+    uint32_t cex = dc;
+    block_excl_scan(mex, cex, S);
+    U128 before = bs;
+    u128_add(before, mex);
+    U128 after = before;
+    u128_add(after, dm);
+    if (tid == 0) S.found = 0;
+    __syncthreads();
+    if (tid < 256 && dc > 0u && !certified128(Z, before, eps) && certified128(Z, after, eps)) {
+      S.jstar = 255 - tid;
+      S.cum = before;
+      S.cabove = above + cex;  // window keys ranked above this digit
+      S.found = 1;
+    }
+    __syncthreads();
+    if (!S.found) {
+      ok = false;
+      break;
+    }
+    prefix = (prefix << 8) | (unsigned long long)S.jstar;
+    bs = S.cum;
+    above = S.cabove;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    if (!ok) {
+      atomicOr(status, CTA_DEV_NONFINITE);  // only rows with non-finite weights get here
+      prefix = 0ull;
+    }
+    S.cut = prefix;
+    U128 c = bs;
+    u128_add(c, mass62(weight(ck_logit(prefix), M, sc)));
+    S.C = c;
+    S.k = (long long)NH + above + 1;
+  }
+  __syncthreads();
+}
+
+// Partial sums of a segment's window keys (kept and dropped), their fp64
+// weight sums and largest dropped logit, and the running output position.
+struct WinSums {
+  float ah[4], at[4];
+  double whw, wtw;
+  float dmx;
+  uint32_t pos_out;
+};
+
+// Cold path of a segment (no usable candidate list): the segment's logits are
+// scanned chunk by chunk; kept keys' indices are written in order and the
+// window keys' value rows gathered through per-warp lists.
+template <bool ERR>
+__device__ __noinline__ WinSums settle_scan_segment(const float* __restrict__ ur,
+                                                    const __nv_bfloat16* __restrict__ Vg,
+                                                    int32_t* __restrict__ dst, int64_t n,
+                                                    int64_t k_lo, int64_t k_hi, float M, float sc,
+                                                    int llo, int lhi, uint32_t cut_key,
+                                                    uint32_t cut_idx, uint32_t pos_out,
+                                                    SettleShared& S) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float ah[4] = {0.f, 0.f, 0.f, 0.f}, at[4] = {0.f, 0.f, 0.f, 0.f};
+  double whw = 0.0, wtw = 0.0;
+  float dmx = kNegInf;
+  auto gather_list = [&](const unsigned long long* keys, const unsigned char* kept, int first,
+                         int end, int stride) {
+    for (int e0 = first; e0 < end; e0 += 8 * stride) {
+      uint2 v[8];
+      float w8[8];
+      int kp[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int e = e0 + q * stride;
+        kp[q] = -1;
+        w8[q] = 0.0f;
+        v[q] = make_uint2(0u, 0u);
+        if (e < end) {
+          const unsigned long long lk = keys[e];
+          const float x = __uint_as_float((uint32_t)(lk >> 32));
+          w8[q] = weight(x, M, sc);
+          kp[q] = kept[e];
+          v[q] = __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)(uint32_t)lk * kTD) + lane);
+          if (!kp[q]) dmx = fmaxf(dmx, x);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (kp[q] < 0) continue;
+        const float2 a = bf16x2_to_float2(v[q].x), b = bf16x2_to_float2(v[q].y);
+        if (kp[q]) {
+          ah[0] = fmaf(w8[q], a.x, ah[0]);
+          ah[1] = fmaf(w8[q], a.y, ah[1]);
+          ah[2] = fmaf(w8[q], b.x, ah[2]);
+          ah[3] = fmaf(w8[q], b.y, ah[3]);
+          whw += (double)w8[q];
+        } else {
+          if constexpr (ERR) {
+            at[0] = fmaf(w8[q], a.x, at[0]);
+            at[1] = fmaf(w8[q], a.y, at[1]);
+            at[2] = fmaf(w8[q], b.x, at[2]);
+            at[3] = fmaf(w8[q], b.y, at[3]);
+          }
+          wtw += (double)w8[q];
+        }
+      }
+    }
+    __syncwarp();
+  };
+  int nl = 0;  // entries in this warp's window list (warp-uniform)
+  unsigned long long* wlk = S.wl_key[warp];
+  unsigned char* wlf = S.wl_kept[warp];
+  auto drain = [&]() {
+    gather_list(wlk, wlf, 0, nl, 1);
+    nl = 0;
+  };
+for (int64_t b0 = k_lo; b0 < k_hi; b0 += (int64_t)kBatch * kChunk) {
+  float4 xv[kBatch];
+#pragma unroll
+  for (int c = 0; c < kBatch; ++c) {
+    const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
+    // rows of the logits are padded to a multiple of 64 keys: the 16-byte
+    // load of four keys starting below k_hi stays inside the row
+    xv[c] = key0 < k_hi ? __ldcg(reinterpret_cast<const float4*>(ur + key0))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  uint32_t kbits = 0u, wbits = 0u;  // bit 4c + e: key e of chunk c kept / in the window
+  unsigned long long pk[2] = {0ull, 0ull};
+#pragma unroll
+  for (int c = 0; c < kBatch; ++c) {
+    const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
+    const float xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const bool valid = key0 + e < k_hi;
+      const uint32_t ok = order_key(xs[e]);
+      // kept iff the composite key is >= the cut's (a key outside the
+      // window lies on the side of the cut that its bracket side names)
+      if (valid && (ok > cut_key || (ok == cut_key && (uint32_t)(key0 + e) <= cut_idx)))
+        kbits |= 1u << (4 * c + e);
+      const bool win = in_window(xs[e], sc, llo, lhi);
+      if (valid && win) wbits |= 1u << (4 * c + e);
+    }
+    pk[c >> 2] += (unsigned long long)__popc((kbits >> (4 * c)) & 0xfu) << (16 * (c & 3));
+  }
+  unsigned long long tot[2];
+  block_excl_scan_packed(pk, tot, S);
+  uint32_t chunk_base = pos_out;
+#pragma unroll
+  for (int c = 0; c < kBatch; ++c) {
+    const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
+    const uint32_t kb = (kbits >> (4 * c)) & 0xfu;
+    uint32_t at_ = chunk_base + (uint32_t)((pk[c >> 2] >> (16 * (c & 3))) & 0xffffull);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if ((kb >> e) & 1u) {
+        if (at_ < (uint32_t)n) dst[at_] = (int32_t)(key0 + e);
+        ++at_;
+      }
+    }
+    chunk_base += (uint32_t)((tot[c >> 2] >> (16 * (c & 3))) & 0xffffull);
+    // window keys of the chunk to this warp's list
+    const uint32_t wb = (wbits >> (4 * c)) & 0xfu;
+    if (__any_sync(0xffffffffu, wb != 0u)) {
+      const uint32_t cnt = __popc(wb);
+      uint32_t pre = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += y;
+      }
+      const int total = (int)__shfl_sync(0xffffffffu, pre, 31);
+      int slot = nl + (int)(pre - cnt);
+      const float xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if ((wb >> e) & 1u) {
+          wlk[slot] = ((unsigned long long)__float_as_uint(xs[e]) << 32) | (uint32_t)(key0 + e);
+          wlf[slot] = (unsigned char)((kb >> e) & 1u);
+          ++slot;
+        }
+      }
+      __syncwarp();
+      nl += total;
+      if (nl > kWList - 4 * kWarp) drain();  // the next chunk may add 128
+    }
+  }
+  pos_out = chunk_base;
+}
+  if (nl) drain();
+  WinSums r;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    r.ah[i] = ah[i];
+    r.at[i] = at[i];
+  }
+  r.whw = whw;
+  r.wtw = wtw;
+  r.dmx = dmx;
+  r.pos_out = pos_out;
+  return r;
+}
+
 template <bool ERR>
 __global__ void __launch_bounds__(kTThreads, 2)
 settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ u, TcBufs tb,
@@ -260,13 +550,18 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
   const int64_t seg_lo = (int64_t)r_first * p.rstages * 128;
   const int64_t seg_hi = min(n, (int64_t)r_last * p.rstages * 128);
   const int64_t mw_lo = seg_lo >> 5, mw_hi = (seg_hi + 31) >> 5;  // 4-word aligned
-  {
-    const unsigned long long* cand = tb.cand + row * kCandCap;
-    for (int i = tid; i < kCandCap / 2; i += kTThreads) cp_async16(&S.cand[2 * i], cand + 2 * i);
-    const uint32_t* hm = tb.hmask + row * tb.mask_words + mw_lo;
-    const int nw0 = (int)min((int64_t)kMaskBlock, mw_hi - mw_lo);
-    for (int i = tid; 4 * i < nw0; i += kTThreads) cp_async16(&S.mask0[4 * i], hm + 4 * i);
-    cp_async_commit();
+  // (bulk copies on the barrier bar_in, issued by one thread; a candidate
+  // list or mask row starts on a 16-byte boundary and the copied mask words
+  // are whole groups of four, inside the row)
+  if (tid == 0) {
+    mbar_init(&S.bar_in, 1);
+    mbar_init(&S.bar_v, 1);
+    mbar_fence_init();
+    const unsigned long long pol = policy_evict_first();
+    const unsigned nb0 = 16u * (unsigned)((min((int64_t)kMaskBlock, mw_hi - mw_lo) + 3) / 4);
+    mbar_arrive_expect_tx(&S.bar_in, (unsigned)(kCandCap * 8) + nb0);
+    bulk_load(S.cand, tb.cand + row * kCandCap, (unsigned)(kCandCap * 8), &S.bar_in, pol);
+    if (nb0) bulk_load(S.mask0, tb.hmask + row * tb.mask_words + mw_lo, nb0, &S.bar_in, pol);
   }
   // ---- 1. row totals (warp 0: one range record per lane) ----------------------
   if (warp == 0) {
@@ -335,12 +630,13 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
     S.found = 0;
     S.nlist = 0u;
   }
-  cp_async_wait<0>();
+  if (!mbar_wait(&S.bar_in, 0u) && tid == 0) atomicOr(status, CTA_DEV_TIMEOUT);
   __syncthreads();
   // fast path: the segment's window keys (the candidates with an index in
   // it) to a flat list, and the value rows of the first kVPre of them copied
   // in while the cut is searched
   unsigned long long* fl_key = &S.wl_key[0][0];  // flat list of kTWarps * kWList entries
+  int vcopies = 0;  // value rows in flight on bar_v (waited for on every path)
   if (fast) {
     for (int i = tid; i < m; i += kTThreads) {
       const unsigned long long ck = S.cand[i];
@@ -352,13 +648,17 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
     }
     __syncthreads();
     const int npre = min((int)S.nlist, kVPre);
-    const __nv_bfloat16* Vr = V + (row / p.gm) * n * kTD;
-    for (int i = tid; i < npre * (kTD / 8); i += kTThreads) {  // 16 pieces of 16 B per row
-      const int e = i / (kTD / 8), c = i % (kTD / 8);
-      const uint32_t idx = 0xffffffffu - (uint32_t)(fl_key[e] & 0xffffffffull);
-      cp_async16(&S.vrow[e][2 * c], Vr + (int64_t)idx * kTD + 8 * c);
+    vcopies = npre;
+    if (warp == 0 && npre > 0) {  // one 256-byte bulk copy per row, on bar_v
+      const __nv_bfloat16* Vr = V + (row / p.gm) * n * kTD;
+      const unsigned long long pol = policy_evict_first();
+      if (lane == 0) mbar_arrive_expect_tx(&S.bar_v, (unsigned)npre * (unsigned)(kTD * 2));
+      __syncwarp();
+      for (int e = lane; e < npre; e += kWarp) {
+        const uint32_t idx = 0xffffffffu - (uint32_t)(fl_key[e] & 0xffffffffull);
+        bulk_load(&S.vrow[e][0], Vr + (int64_t)idx * kTD, (unsigned)(kTD * 2), &S.bar_v, pol);
+      }
     }
-    cp_async_commit();
   }
 
   // ---- 2. the exact cut --------------------------------------------------------
@@ -463,120 +763,12 @@ settle_tc_kernel(const __nv_bfloat16* __restrict__ V, const float* __restrict__ 
   }
 full_sort:
   if (fast && !S.found) {
-    // the whole candidate list sorted, then walked from the top
-    int P = 1;
-    while (P < m) P <<= 1;
-    for (int i = m + tid; i < P; i += kTThreads) S.cand[i] = 0ull;  // pad below all keys
-    __syncthreads();
-    bitonic_sort_desc(S.cand, P);
-    constexpr int E = kCandCap / kTThreads;
-    unsigned long long Wl[E];
-    U128 ls = u128_zero();
-#pragma unroll
-    for (int j = 0; j < E; ++j) {
-      const int i = tid * E + j;
-      Wl[j] = (i < m) ? mass62(weight(ck_logit(S.cand[i]), M, sc)) : 0ull;
-      u128_add(ls, Wl[j]);
-    }
-    U128 cum = ls;
-    uint32_t dummy = 0u;
-    block_excl_scan(cum, dummy, S);
-    u128_add(cum, base);
-    U128 end = cum;
-    u128_add(end, ls);
-    if (!certified128(Z, cum, eps) && certified128(Z, end, eps)) {
-#pragma unroll
-      for (int j = 0; j < E; ++j) {
-        const int i = tid * E + j;
-        U128 nx = cum;
-        u128_add(nx, Wl[j]);
-        if (i < m && certified128(Z, nx, eps)) {
-          S.C = nx;
-          S.cut = S.cand[i];
-          S.k = (long long)NH + i + 1;
-          S.found = 1;
-          break;
-        }
-        cum = nx;
-      }
-    }
-    __syncthreads();
-    if (!S.found) {  // excluded by the checks above; recompute by the radix path
+    if (!cut_by_sort(S, m, M, sc, NH, Z, base, eps)) {
       if (tid == 0 && seg == 0) atomicOr(status, CTA_DEV_INTERNAL);
       fast = false;
     }
   }
-  if (!fast) {
-    // radix select over the window's composite keys, eight bits per pass
-    unsigned long long prefix = 0ull;
-    U128 bs = base;
-    uint32_t above = 0u;
-    bool ok = true;
-    for (int level = 0; level < 8 && ok; ++level) {
-      const int shift = 56 - 8 * level;
-      for (int i = tid; i < 256; i += kTThreads) {
-        S.u.rx.lo[i] = 0ull;
-        S.u.rx.hi[i] = 0ull;
-        S.u.rx.cnt[i] = 0u;
-      }
-      __syncthreads();
-      for (int64_t key = tid; key < n; key += kTThreads) {
-        const float x = __ldcg(ur + key);
-        if (!in_window(x, sc, llo, lhi)) continue;
-        const unsigned long long ck = composite(order_key(x), (uint32_t)key);
-        if (level > 0 && (ck >> (64 - 8 * level)) != prefix) continue;
-        const int dig = (int)((ck >> shift) & 0xffull);
-        const unsigned long long w = mass62(weight(x, M, sc));
-        const unsigned long long old = atomicAdd(&S.u.rx.lo[dig], w);
-        if (old + w < old) atomicAdd(&S.u.rx.hi[dig], 1ull);
-        atomicAdd(&S.u.rx.cnt[dig], 1u);
-      }
-      __syncthreads();
-      // digits in descending order: thread t < 256 owns digit 255 - t
-      U128 dm = u128_zero();
-      uint32_t dc = 0u;
-      if (tid < 256) {
-        dm = u128_make(S.u.rx.lo[255 - tid], S.u.rx.hi[255 - tid]);
-        dc = S.u.rx.cnt[255 - tid];
-      }
-      U128 mex = dm;
-      uint32_t cex = dc;
-      block_excl_scan(mex, cex, S);
-      U128 before = bs;
-      u128_add(before, mex);
-      U128 after = before;
-      u128_add(after, dm);
-      if (tid == 0) S.found = 0;
-      __syncthreads();
-      if (tid < 256 && dc > 0u && !certified128(Z, before, eps) && certified128(Z, after, eps)) {
-        S.jstar = 255 - tid;
-        S.cum = before;
-        S.cabove = above + cex;  // window keys ranked above this digit
-        S.found = 1;
-      }
-      __syncthreads();
-      if (!S.found) {
-        ok = false;
-        break;
-      }
-      prefix = (prefix << 8) | (unsigned long long)S.jstar;
-      bs = S.cum;
-      above = S.cabove;
-      __syncthreads();
-    }
-    if (tid == 0) {
-      if (!ok) {
-        atomicOr(status, CTA_DEV_NONFINITE);  // only rows with non-finite weights get here
-        prefix = 0ull;
-      }
-      S.cut = prefix;
-      U128 c = bs;
-      u128_add(c, mass62(weight(ck_logit(prefix), M, sc)));
-      S.C = c;
-      S.k = (long long)NH + above + 1;
-    }
-    __syncthreads();
-  }
+  if (!fast) cut_by_radix(S, ur, n, M, sc, llo, lhi, NH, Z, base, eps, status);
   const unsigned long long cut = S.cut;
   const uint32_t cut_key = (uint32_t)(cut >> 32);
   const uint32_t cut_idx = 0xffffffffu - (uint32_t)(cut & 0xffffffffull);
@@ -620,97 +812,37 @@ full_sort:
     float dmx = kNegInf;
     // value rows of listed window keys: entries first, first + stride, ...
     // below end, eight loads in flight per round (whole warp)
-    auto gather_list = [&](const unsigned long long* keys, const unsigned char* kept, int first,
-                           int end, int stride) {
-      for (int e0 = first; e0 < end; e0 += 8 * stride) {
-        uint2 v[8];
-        float w8[8];
-        int kp[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int e = e0 + q * stride;
-          kp[q] = -1;
-          w8[q] = 0.0f;
-          v[q] = make_uint2(0u, 0u);
-          if (e < end) {
-            const unsigned long long lk = keys[e];
-            const float x = __uint_as_float((uint32_t)(lk >> 32));
-            w8[q] = weight(x, M, sc);
-            kp[q] = kept[e];
-            v[q] = __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)(uint32_t)lk * kTD) + lane);
-            if (!kp[q]) dmx = fmaxf(dmx, x);
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (kp[q] < 0) continue;
-          const float2 a = bf16x2_to_float2(v[q].x), b = bf16x2_to_float2(v[q].y);
-          if (kp[q]) {
-            ah[0] = fmaf(w8[q], a.x, ah[0]);
-            ah[1] = fmaf(w8[q], a.y, ah[1]);
-            ah[2] = fmaf(w8[q], b.x, ah[2]);
-            ah[3] = fmaf(w8[q], b.y, ah[3]);
-            whw += (double)w8[q];
-          } else {
-            if constexpr (ERR) {
-              at[0] = fmaf(w8[q], a.x, at[0]);
-              at[1] = fmaf(w8[q], a.y, at[1]);
-              at[2] = fmaf(w8[q], b.x, at[2]);
-              at[3] = fmaf(w8[q], b.y, at[3]);
-            }
-            wtw += (double)w8[q];
-          }
-        }
-      }
-      __syncwarp();
-    };
     if (fast) {
       // The window keys of the segment are the candidates with an index in it
       // (the flat list); every other key's side is in the value pass's
       // kept-for-certain mask.  The first kVPre value rows are in shared memory.
       const int nlist = (int)S.nlist;
-      cp_async_wait<0>();
-      __syncthreads();
-      for (int e0 = warp; e0 < nlist; e0 += 8 * kTWarps) {
-        uint2 v[8];
-        float w8[8];
-        int kp[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int e = e0 + q * kTWarps;
-          kp[q] = -1;
-          w8[q] = 0.0f;
-          v[q] = make_uint2(0u, 0u);
-          if (e < nlist) {
-            const unsigned long long ck = fl_key[e];
-            const float x = ck_logit(ck);
-            const uint32_t idx = 0xffffffffu - (uint32_t)(ck & 0xffffffffull);
-            w8[q] = weight(x, M, sc);
-            kp[q] = ck >= cut ? 1 : 0;
-            v[q] = e < kVPre ? S.vrow[e][lane]
-                             : __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)idx * kTD) + lane);
-            if (!kp[q]) dmx = fmaxf(dmx, x);
+      if (vcopies > 0 && !mbar_wait(&S.bar_v, 0u) && tid == 0) atomicOr(status, CTA_DEV_TIMEOUT);
+      // one entry per warp and step (a short loop body: this code runs once per
+      // CTA, so its size rather than its latency decides)
+      for (int e = warp; e < nlist; e += kTWarps) {
+        const unsigned long long ck = fl_key[e];
+        const float x = ck_logit(ck);
+        const uint32_t idx = 0xffffffffu - (uint32_t)(ck & 0xffffffffull);
+        const float w = weight(x, M, sc);
+        const uint2 vv = e < kVPre ? S.vrow[e][lane]
+                                   : __ldg(reinterpret_cast<const uint2*>(Vg + (int64_t)idx * kTD) + lane);
+        const float2 a = bf16x2_to_float2(vv.x), b = bf16x2_to_float2(vv.y);
+        if (ck >= cut) {
+          ah[0] = fmaf(w, a.x, ah[0]);
+          ah[1] = fmaf(w, a.y, ah[1]);
+          ah[2] = fmaf(w, b.x, ah[2]);
+          ah[3] = fmaf(w, b.y, ah[3]);
+          whw += (double)w;
+        } else {
+          if constexpr (ERR) {
+            at[0] = fmaf(w, a.x, at[0]);
+            at[1] = fmaf(w, a.y, at[1]);
+            at[2] = fmaf(w, b.x, at[2]);
+            at[3] = fmaf(w, b.y, at[3]);
           }
-        }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (kp[q] < 0) continue;
-          const float2 a = bf16x2_to_float2(v[q].x), b = bf16x2_to_float2(v[q].y);
-          if (kp[q]) {
-            ah[0] = fmaf(w8[q], a.x, ah[0]);
-            ah[1] = fmaf(w8[q], a.y, ah[1]);
-            ah[2] = fmaf(w8[q], b.x, ah[2]);
-            ah[3] = fmaf(w8[q], b.y, ah[3]);
-            whw += (double)w8[q];
-          } else {
-            if constexpr (ERR) {
-              at[0] = fmaf(w8[q], a.x, at[0]);
-              at[1] = fmaf(w8[q], a.y, at[1]);
-              at[2] = fmaf(w8[q], b.x, at[2]);
-              at[3] = fmaf(w8[q], b.y, at[3]);
-            }
-            wtw += (double)w8[q];
-          }
+          wtw += (double)w;
+          dmx = fmaxf(dmx, x);
         }
       }
       // kept indices: mask words of the segment, in blocks of kMaskBlock words
@@ -751,99 +883,68 @@ full_sort:
         }
         if (tid == kTThreads - 1) S.off_win = o;  // the block's kept keys
         __syncthreads();
-        // one 32-key word per warp step: coalesced index writes
-        for (int wi = warp; wi < nwb; wi += kTWarps) {
-          const uint32_t bits = S.u.mk.word[wi];
-          if ((bits >> lane) & 1u) {
-            const uint32_t at_ = pos_out + S.u.mk.off[wi] + __popc(bits & ((1u << lane) - 1u));
-            if (at_ < (uint32_t)n) dst[at_] = (int32_t)(((wb0 + wi) << 5) + lane);
+        // The block's indices go out through shared memory, kStageWords words
+        // at a time: compacted there (the candidate list is no longer read),
+        // index i at slot i - g0 + pad so that a 16-byte boundary of idx_out is
+        // one of the staging area; the aligned middle goes out as one bulk
+        // copy, the (at most three) indices at either end as plain stores.
+        int* stage = reinterpret_cast<int*>(S.cand);
+        const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(dst) >> 2) & 3u;
+        for (int s0 = 0; s0 < nwb; s0 += kStageWords) {
+          const int s1 = min(nwb, s0 + kStageWords);
+          const uint32_t off0 = S.u.mk.off[s0];
+          const uint32_t off1 = s1 < nwb ? S.u.mk.off[s1] : S.off_win;
+          // global positions [g0, g1) (never past n, whatever the records say)
+          const uint32_t g0 = min(pos_out + off0, (uint32_t)n);
+          const uint32_t g1 = min(pos_out + off1, (uint32_t)n);
+          const uint32_t pad = (g0 + mis) & 3u;
+          for (int w0 = s0 + warp; w0 < s1; w0 += 4 * kTWarps) {
+            uint32_t bits[4], off[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int wi = w0 + q * kTWarps;
+              bits[q] = wi < s1 ? S.u.mk.word[wi] : 0u;
+              off[q] = wi < s1 ? S.u.mk.off[wi] : 0u;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              if ((bits[q] >> lane) & 1u)  // slot < kStageWords * 32 + 3
+                stage[pad + off[q] - off0 + __popc(bits[q] & ((1u << lane) - 1u))] =
+                    (int)(((wb0 + w0 + q * kTWarps) << 5) + lane);
+            }
           }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // staged indices -> bulk copy
+          __syncthreads();
+          uint32_t a0 = g0 + ((4u - pad) & 3u);  // first 16-byte boundary
+          uint32_t a1 = g1;
+          if (a0 >= g1 || g1 - a0 < 4u)
+            a0 = g1;  // short: plain stores only
+          else
+            a1 = g1 - ((g1 + mis) & 3u);  // last 16-byte boundary, >= a0
+          for (uint32_t i = g0 + tid; i < a0; i += kTThreads) dst[i] = stage[i - g0 + pad];
+          for (uint32_t i = a1 + tid; i < g1; i += kTThreads) dst[i] = stage[i - g0 + pad];
+          if (tid == 0 && a1 > a0) {
+            bulk_store(dst + a0, stage + (a0 - g0 + pad), (a1 - a0) * 4u);
+            bulk_commit();
+            bulk_wait_read();  // the staging area may be written again
+          }
+          __syncthreads();
         }
         pos_out += S.off_win;
         __syncthreads();
       }
     } else {
-      int nl = 0;  // entries in this warp's window list (warp-uniform)
-      unsigned long long* wlk = S.wl_key[warp];
-      unsigned char* wlf = S.wl_kept[warp];
-      auto drain = [&]() {
-        gather_list(wlk, wlf, 0, nl, 1);
-        nl = 0;
-      };
-    for (int64_t b0 = k_lo; b0 < k_hi; b0 += (int64_t)kBatch * kChunk) {
-      float4 xv[kBatch];
+      const WinSums w = settle_scan_segment<ERR>(ur, Vg, dst, n, k_lo, k_hi, M, sc, llo, lhi,
+                                                 cut_key, cut_idx, pos_out, S);
 #pragma unroll
-      for (int c = 0; c < kBatch; ++c) {
-        const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
-        // rows of the logits are padded to a multiple of 64 keys: the 16-byte
-        // load of four keys starting below k_hi stays inside the row
-        xv[c] = key0 < k_hi ? __ldcg(reinterpret_cast<const float4*>(ur + key0))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i = 0; i < 4; ++i) {
+        ah[i] += w.ah[i];
+        at[i] += w.at[i];
       }
-      uint32_t kbits = 0u, wbits = 0u;  // bit 4c + e: key e of chunk c kept / in the window
-      unsigned long long pk[2] = {0ull, 0ull};
-#pragma unroll
-      for (int c = 0; c < kBatch; ++c) {
-        const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
-        const float xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool valid = key0 + e < k_hi;
-          const uint32_t ok = order_key(xs[e]);
-          // kept iff the composite key is >= the cut's (a key outside the
-          // window lies on the side of the cut that its bracket side names)
-          if (valid && (ok > cut_key || (ok == cut_key && (uint32_t)(key0 + e) <= cut_idx)))
-            kbits |= 1u << (4 * c + e);
-          const bool win = in_window(xs[e], sc, llo, lhi);
-          if (valid && win) wbits |= 1u << (4 * c + e);
-        }
-        pk[c >> 2] += (unsigned long long)__popc((kbits >> (4 * c)) & 0xfu) << (16 * (c & 3));
-      }
-      unsigned long long tot[2];
-      block_excl_scan_packed(pk, tot, S);
-      uint32_t chunk_base = pos_out;
-#pragma unroll
-      for (int c = 0; c < kBatch; ++c) {
-        const int64_t key0 = b0 + (int64_t)c * kChunk + 4 * tid;
-        const uint32_t kb = (kbits >> (4 * c)) & 0xfu;
-        uint32_t at_ = chunk_base + (uint32_t)((pk[c >> 2] >> (16 * (c & 3))) & 0xffffull);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((kb >> e) & 1u) {
-            if (at_ < (uint32_t)n) dst[at_] = (int32_t)(key0 + e);
-            ++at_;
-          }
-        }
-        chunk_base += (uint32_t)((tot[c >> 2] >> (16 * (c & 3))) & 0xffffull);
-        // window keys of the chunk to this warp's list
-        const uint32_t wb = (wbits >> (4 * c)) & 0xfu;
-        if (__any_sync(0xffffffffu, wb != 0u)) {
-          const uint32_t cnt = __popc(wb);
-          uint32_t pre = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, pre, o);
-            if (lane >= o) pre += y;
-          }
-          const int total = (int)__shfl_sync(0xffffffffu, pre, 31);
-          int slot = nl + (int)(pre - cnt);
-          const float xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if ((wb >> e) & 1u) {
-              wlk[slot] = ((unsigned long long)__float_as_uint(xs[e]) << 32) | (uint32_t)(key0 + e);
-              wlf[slot] = (unsigned char)((kb >> e) & 1u);
-              ++slot;
-            }
-          }
-          __syncwarp();
-          nl += total;
-          if (nl > kWList - 4 * kWarp) drain();  // the next chunk may add 128
-        }
-      }
-      pos_out = chunk_base;
-    }
-      if (nl) drain();
+      whw += w.whw;
+      wtw += w.wtw;
+      dmx = fmaxf(dmx, w.dmx);
+      pos_out = w.pos_out;
     }
     // ---- the range's results: value pass partial + window sums -------------------
 #pragma unroll
@@ -903,6 +1004,8 @@ full_sort:
   }
 
   // ---- 4. the row's last CTA forms the outputs ------------------------------------
+  if (vcopies > 0) mbar_wait(&S.bar_v, 0u);  // no copy into this CTA is left in flight
+  if (tid == 0) bulk_wait_all();             // the bulk index stores are done
   __threadfence();
   __syncthreads();
   if (tid == 0) S.last = atomicAdd(tb.ticket + row, 1u) == (uint32_t)(nseg - 1);

@@ -79,9 +79,13 @@ typedef struct {
   float* kl_out;          /* [batch, n_heads, m] KL(P-hat || P) = log(sum_all w / sum_head w)
                              from the output pass, or NULL                                   */
   uint32_t* status_dev;   /* device word for CTA_DEV_* bits, or NULL                         */
-  void** phase_events;    /* NULL, or 5 cudaEvent_t recorded on the stream before the score
-                             phase, after it, after selection, after the output pass and
-                             after finalisation (for timing individual phases)                */
+  void** phase_events;    /* NULL, or 5 cudaEvent_t recorded on the stream (for timing the
+                             kernels one by one; an event between two kernels keeps the second
+                             from starting early).  bf16 with d = 128 (the tensor-core decode
+                             path): before the logits pass, after it, after the row brackets,
+                             after the value pass and after the last kernel (cut, indices,
+                             outputs).  Other shapes: before the score phase, after it, after
+                             selection, after the output pass and after finalisation.          */
   float* gap_out;         /* [batch, n_heads, m] single-gap certificate, or NULL: with
                              u_(k) the last kept and u_(k+1) the largest dropped logit,
                              1 / (1 + k/(n-k) exp((u_(k) - u_(k+1)) / sqrt(d))), an upper
