@@ -65,7 +65,8 @@ constexpr int kMaskBlock = 4 * kTThreads;  // mask words per block of the index 
 constexpr int kVPre = 128;
 constexpr int kStageWords = 124;         // mask words per staging round (124 x 32 + 3 <= 4096 slots)               // window value rows copied in while the cut is searched
 
-static_assert(kCandCap * 2 >= kStageWords * 32 + 3, "the candidate list doubles as the staging area");
+static_assert(kCandCap * 2 >= kStageWords * 32 + 3 && kVPre * kTD / 2 >= kStageWords * 32 + 3,
+              "the candidate list and the window rows double as the staging areas");
 
 struct SettleShared {
   alignas(16) unsigned long long cand[kCandCap];  // the row's candidates (sorted in place by the fallback)
@@ -115,6 +116,9 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -888,9 +892,16 @@ full_sort:
         // index i at slot i - g0 + pad so that a 16-byte boundary of idx_out is
         // one of the staging area; the aligned middle goes out as one bulk
         // copy, the (at most three) indices at either end as plain stores.
-        int* stage = reinterpret_cast<int*>(S.cand);
+        // Two staging areas take turns (the candidate list and the window
+        // rows, both read by now), so that a round's compaction overlaps the
+        // previous round's bulk copy.
         const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(dst) >> 2) & 3u;
-        for (int s0 = 0; s0 < nwb; s0 += kStageWords) {
+        for (int s0 = 0, rnd = 0; s0 < nwb; s0 += kStageWords, ++rnd) {
+          int* stage = (rnd & 1) ? reinterpret_cast<int*>(&S.vrow[0][0]) : reinterpret_cast<int*>(S.cand);
+          if (rnd >= 2) {  // this area's copy of two rounds ago has read it
+            if (tid == 0) bulk_wait_read1();
+            __syncthreads();
+          }
           const int s1 = min(nwb, s0 + kStageWords);
           const uint32_t off0 = S.u.mk.off[s0];
           const uint32_t off1 = s1 < nwb ? S.u.mk.off[s1] : S.off_win;
@@ -923,13 +934,13 @@ full_sort:
             a1 = g1 - ((g1 + mis) & 3u);  // last 16-byte boundary, >= a0
           for (uint32_t i = g0 + tid; i < a0; i += kTThreads) dst[i] = stage[i - g0 + pad];
           for (uint32_t i = a1 + tid; i < g1; i += kTThreads) dst[i] = stage[i - g0 + pad];
-          if (tid == 0 && a1 > a0) {
-            bulk_store(dst + a0, stage + (a0 - g0 + pad), (a1 - a0) * 4u);
-            bulk_commit();
-            bulk_wait_read();  // the staging area may be written again
+          if (tid == 0) {
+            if (a1 > a0) bulk_store(dst + a0, stage + (a0 - g0 + pad), (a1 - a0) * 4u);
+            bulk_commit();  // one group per round (possibly empty)
           }
-          __syncthreads();
         }
+        if (tid == 0) bulk_wait_read();  // both areas may be written again
+        __syncthreads();
         pos_out += S.off_win;
         __syncthreads();
       }
