@@ -25,14 +25,13 @@
  *     argument and launch errors only.  Conditions found on the device (a
  *     non-finite logit, a broken internal invariant) are OR-ed as bits into
  *     *cta_opts.status_dev when that pointer is given.  No device code traps.
- *   - For bf16 inputs with d = 128 the kernels of a call are launched with
- *     programmatic stream serialization: the first one may start reading q
- *     and K while the kernel before it on the stream finishes, if that kernel
- *     lets its dependents launch early (griddepcontrol.launch_dependents);
- *     it writes nothing before that kernel has completed.  A caller's kernel
- *     that triggers its dependents early must not write q or K after the
- *     trigger.  Kernels that never trigger (the usual case) and copies give
- *     ordinary stream order.
+ *   - For bf16 inputs with d = 128 the four kernels of a call are launched
+ *     with programmatic stream serialization (each may become resident while
+ *     the one before it finishes).  The first waits for the kernel before it
+ *     on the stream to complete (griddepcontrol.wait) before it reads q or K
+ *     or writes anything; V is read only after the first has completed.  So a
+ *     caller's kernel that writes q, K or V right before the call is ordered
+ *     before every read, whether or not it triggers its dependents early.
  *   - Supported: d in {64, 128}; 1 <= n <= 2^28; 0 < eps < 1;
  *     n_heads % n_kv_heads == 0; batch, m >= 1.  There is no mask: every row
  *     sees all n keys.  The logit scale is 1/sqrt(d).
@@ -104,7 +103,9 @@ void cta_opts_init(cta_opts* o);
  * Bytes of device workspace cta_certified_topk_attn needs for this shape
  * (batch, m and dtype are taken from o; NULL = defaults).  Returns 0 for an
  * unsupported shape.  The workspace holds the fp32 logits of every row
- * (4 * rows * n bytes) plus small per-row and per-chunk records.
+ * (4 * rows * n bytes) plus per-row and per-range records; for bf16 with
+ * d = 128 also per-range level histograms (6.6 KB per row and key range),
+ * a candidate list per row (16 KB) and one bit per key and row.
  */
 size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const cta_opts* o);
 
@@ -129,9 +130,12 @@ size_t cta_workspace_size(int64_t n, int d, int n_heads, int n_kv_heads, const c
  *
  * Numerics: logits are fp32 dot products (bf16 inputs widen exactly); the
  * ranking uses them.  Softmax numerators w_i = exp(s_i - max s) are fp32 and
- * are summed exactly as 64-bit fixed-point integers, so the k_eps decision,
- * TV and the kept set do not depend on the reduction order; the decision is
- * taken in fp64 as (Z - C_k) / Z <= eps.  Output sums accumulate in fp32 over
+ * are summed exactly as fixed-point integers (units of 2^-62 in 128-bit sums
+ * for bf16 with d = 128; otherwise a 64-bit scale chosen per row from its
+ * mass), so the k_eps decision, TV and the kept set do not depend on the
+ * reduction order and the rounding of the n numerators moves the total by
+ * at most n * 2^-62 of it; the decision is taken in fp64 as
+ * (Z - C_k) / Z <= eps.  Output sums accumulate in fp32 over
  * short runs and in fp64 across them.  Results are bit-reproducible.
  * Returns a cta_status.
  */
