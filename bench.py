@@ -38,7 +38,12 @@ sys.path.insert(0, ROOT)
 METRIC = "certified top-k attn query-heads/s & HBM GB/s (% of peak) at n=32K/128K"
 UNIT = "query-heads/s"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ("score_kv_tc.cu", "gather_tc.cu", "settle_tc.cu", "umma.cuh", "common.cuh")
+# the source files of each decode kernel (a profiled traffic figure counts only
+# while these are unchanged since its capture)
+KERNEL_FILES = {"score_kv_tc_kernel": ("score_kv_tc.cu", "common.cuh", "umma.cuh"),
+                "bracket_tc_kernel": ("gather_tc.cu", "common.cuh"),
+                "gather_tc_kernel": ("gather_tc.cu", "common.cuh", "umma.cuh"),
+                "settle_tc_kernel": ("settle_tc.cu", "common.cuh")}
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the measured copy peak is the roofline's denominator)
 # the four kernels of one decode call (bf16 K, V with d = 128), in launch order
 DECODE_PHASES = ("logits", "brackets", "values", "settle")
@@ -99,9 +104,9 @@ def measured_peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in KERNEL_FILES[kernel]:
         with open(os.path.join(ROOT, "certified_top_sparse_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -109,16 +114,16 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(kernel: str):
     """DRAM bytes per launch of `kernel` from the committed ncu summary, or
-    None when it is missing or the kernel sources changed since the capture."""
+    None when it is missing or the kernel's sources changed since the capture."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("source_hash") != kernel_source_hash():
-        return None
     k = rec.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("dram_bytes_per_launch")
+    if k is None or kernel not in KERNEL_FILES or k.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return k.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
