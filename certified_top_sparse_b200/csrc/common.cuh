@@ -226,6 +226,7 @@ struct TcBufs {
   unsigned long long* cand;  // [rows][kCandCap] composite keys of window keys
   uint32_t* cand_cnt;    // [rows] window keys seen (zeroed by the logits pass)
   uint32_t* ticket;      // [rows] ranges settled (zeroed by the logits pass)
+  uint32_t* brk_ready;   // [rows] 1 once the row's bracket is written (zeroed by the logits pass)
   uint32_t* hmask;       // [rows][mask_words] bit j of word w: key 32 w + j kept for certain
   int64_t mask_words;    // words per row: 4 per 128-key stage
 };
@@ -385,12 +386,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned b
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
-}
-
-// Prefetch of global memory into L2 (a hint: no completion, no data returned).
-// src 16-byte aligned; bytes a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -32,7 +32,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 struct Layout {
   size_t u, cmax, sel, choff, acc, gmax, unit, status;
   // tensor-core decode path only (zero-sized otherwise)
-  size_t hist, rrec, srec, brk, cand, cand_cnt, ticket, hmask;
+  size_t hist, rrec, srec, brk, cand, cand_cnt, ticket, brk_ready, hmask;
   size_t total;
 };
 
@@ -126,6 +126,7 @@ Layout layout(const Plan& p, bool tc_decode) {
   L.cand = off;     off = align256(off + sizeof(unsigned long long) * kCandCap * rw);
   L.cand_cnt = off; off = align256(off + sizeof(uint32_t) * rw);
   L.ticket = off;   off = align256(off + sizeof(uint32_t) * rw);
+  L.brk_ready = off; off = align256(off + sizeof(uint32_t) * rw);
   L.hmask = off;    off = align256(off + sizeof(uint32_t) * rw * (size_t)mask_words(p));
   L.total = off;
   return L;
@@ -250,6 +251,7 @@ int cta_certified_topk_attn(const void* q, const void* K, const void* V, int64_t
     tb.cand = reinterpret_cast<unsigned long long*>(ws + L.cand);
     tb.cand_cnt = reinterpret_cast<uint32_t*>(ws + L.cand_cnt);
     tb.ticket = reinterpret_cast<uint32_t*>(ws + L.ticket);
+    tb.brk_ready = reinterpret_cast<uint32_t*>(ws + L.brk_ready);
     tb.hmask = reinterpret_cast<uint32_t*>(ws + L.hmask);
     tb.mask_words = mask_words(p);
     if (launch_score_kv_tc(q, K, u, cmax, tb, p, status, st) != cudaSuccess) return CTA_ERR_CUDA;

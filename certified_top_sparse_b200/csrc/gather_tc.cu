@@ -57,12 +57,12 @@
 // Work items are (KV group, key range, row tile) with ranges cut in stages so
 // that every SM gets about the same number of stages.
 //
-// Ordering: launched as a programmatic dependent of the logits pass.  Its CTAs
-// can start only after every logits CTA has passed its own wait for the
-// caller's preceding kernel, so the value rows may stream at once: the
-// producer fills the first ring of value stages before it waits for the
-// logits pass to complete (griddepcontrol.wait) and only then loads logits.
-// The weight warps wait likewise before they read the histograms.
+// Ordering: logits pass -> bracket kernel -> value pass, each a programmatic
+// dependent of the one before.  The bracket kernel lets the value pass launch
+// only after its own wait for the logits pass, so when a value-pass CTA starts,
+// the logits pass (and the caller's kernels before it) have completed: the
+// producer streams value rows and logits at once, and the weight warps wait
+// only for their own row's bracket (a flag per row, bounded wait).
 #include <algorithm>
 #include <climits>
 
@@ -90,7 +90,6 @@ constexpr int kGEpiThreads = kGWeightWarps * kWarp;  // the weight warps also re
 constexpr int kGEpiBar = 1;           // named barrier of the weight warps
 constexpr uint32_t kGTmemCols = 2 * kGN;
 constexpr int kCandBuf = 128;         // window keys a weight warp buffers (>= 128: one stage's)
-constexpr int kGPrefetch = 12;        // value stages per CTA prefetched into L2 beyond the ring
 constexpr size_t kGSmem = 1024 + (size_t)kGStages * (kGV + kGW + kGU) + kGWeightWarps * kCandBuf * 8;
 static_assert(kGK % 64 == 0 && kGK <= 256, "a stage is whole 64-key swizzle atoms, one TMA box");
 static_assert(kGSmem <= 227 * 1024, "shared memory");
@@ -109,6 +108,38 @@ struct RecPart {
 __device__ __forceinline__ RowBracket ld_cg_bracket(const RowBracket* b) {
   const int4 v = __ldcg(reinterpret_cast<const int4*>(b));
   return RowBracket{__int_as_float(v.x), v.y, v.z, (uint32_t)v.w};
+}
+
+// A row's bracket is handed from the bracket kernel to the value pass through
+// a flag per row (zeroed by the logits pass of the same call): the value pass
+// starts a row as soon as its bracket is out, not when every row's is.
+__device__ __forceinline__ void publish_bracket(RowBracket* b, uint32_t* ready, const RowBracket& v) {
+  *b = v;
+  __threadfence();
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ready), "r"(1u) : "memory");
+}
+// Lane 0 waits (bounded) for the flag; true once it is set.
+__device__ __forceinline__ bool wait_bracket(const uint32_t* ready) {
+  const int lane = threadIdx.x & 31;
+  uint32_t ok = 1u;
+  if (lane == 0) {
+    auto seen = [&]() {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
+      return v != 0u;
+    };
+    if (!seen()) {
+      const unsigned long long t0 = global_ns();
+      ok = 0u;
+      while (global_ns() - t0 <= kWaitLimitNs) {
+        if (seen()) {
+          ok = 1u;
+          break;
+        }
+      }
+    }
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0u;
 }
 
 struct GItem {
@@ -275,7 +306,7 @@ __device__ __forceinline__ void fine_range(const RangeHist* h, int sh, int g0, i
 
 __global__ void __launch_bounds__(kBThreads)
 bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ cmax,
-                  RowBracket* __restrict__ brk, Plan p) {
+                  RowBracket* __restrict__ brk, uint32_t* __restrict__ ready, Plan p) {
   // the histograms and maxima are complete; the value pass may be scheduled
   // from here on (after the logits pass, and so after the caller's kernels)
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -306,7 +337,7 @@ bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ 
   RowBracket out{M, INT_MIN, INT_MAX, 0u};  // default: every key is in the window
   const float XM = __fmul_rn(M, p.scale2);
   if (!(fabsf(XM) < 1.0e6f)) {  // non-finite rows: flagged by the logits pass
-    if (threadIdx.x == 0) brk[row] = out;
+    if (threadIdx.x == 0) publish_bracket(brk + row, ready + row, out);
     return;
   }
   const int T = __float2int_ru(XM) * kLevelsPerOctave;
@@ -329,7 +360,7 @@ bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ 
   deep = warp_sum_f(deep);
   if (lane == 0) s_deep[warp] = deep;
   if (__syncthreads_or(bad)) {
-    if (threadIdx.x == 0) brk[row] = out;
+    if (threadIdx.x == 0) publish_bracket(brk + row, ready + row, out);
     return;
   }
 
@@ -386,7 +417,7 @@ bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ 
   Olo = s_olo;
   Ohi = s_ohi;
   if (Olo <= Ohi) {  // cannot happen with consistent bounds; keep the default
-    if (threadIdx.x == 0) brk[row] = out;
+    if (threadIdx.x == 0) publish_bracket(brk + row, ready + row, out);
     return;
   }
   int g_lo = kLevelsPerOctave * Olo, g_hi = kLevelsPerOctave * Ohi;  // the coarse result
@@ -465,14 +496,14 @@ bracket_tc_kernel(const RangeHist* __restrict__ hist, const float* __restrict__ 
   if (threadIdx.x == 0) {
     out.llo = (Olo > kMergeOct) ? INT_MIN : T - g_lo + 1;
     out.lhi = T - g_hi + 1;
-    brk[row] = out;
+    publish_bracket(brk + row, ready + row, out);
   }
 }
 
 template <int RT, bool ERR>
 __global__ void __launch_bounds__(kGThreads, 1)
 gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restrict__ u,
-                 const unsigned char* __restrict__ vbase, TcBufs tb, float* __restrict__ acc_out, Plan p,
+                 TcBufs tb, float* __restrict__ acc_out, Plan p,
                  uint32_t* __restrict__ status) {
   // the last kernel may be scheduled now; it waits for this grid
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -533,27 +564,20 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<unsigned long long>(&vmap))
                    : "memory");
       // The first ring of value stages goes out at once (the value rows do not
-      // depend on the earlier kernels of the call), and the next kGPrefetch
-      // stages are prefetched into L2 while the brackets are computed.
-      int nA = 0, nP = 0;
-      for (int it = blockIdx.x; it < nitems && nP < kGStages + kGPrefetch; it += gridDim.x) {
+      // depend on the earlier kernels of the call).  (Prefetching the next
+      // 6-24 stages into L2 as well made the step slower.)
+      int nA = 0;
+      for (int it = blockIdx.x; it < nitems && nA < kGStages; it += gridDim.x) {
         const GItem g = gitem_of(it, p);
         const int s_lo = g.range * p.rstages, s_hi = min(spu, s_lo + p.rstages);
-        for (int sg = s_lo; sg < s_hi && nP < kGStages + kGPrefetch; ++sg, ++nP) {
-          if (nA < kGStages) {
-            unsigned char* dst = vring + nA * kGV;
-            mbar_arrive_expect_tx(&vfull[nA], (unsigned)kGV);
-            tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[nA], pol);
-            tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[nA], pol);
-            ++nA;
-          } else {
-            const int64_t key0 = (int64_t)sg * kGK;
-            const unsigned bytes = (unsigned)min((int64_t)kGK, p.n - key0) * (unsigned)(kGD * 2);
-            bulk_prefetch_l2(vbase + ((int64_t)g.group * p.n + key0) * (kGD * 2), bytes);
-          }
+        for (int sg = s_lo; sg < s_hi && nA < kGStages; ++sg, ++nA) {
+          unsigned char* dst = vring + nA * kGV;
+          mbar_arrive_expect_tx(&vfull[nA], (unsigned)kGV);
+          tma_load_3d(dst, &vmap, 0, sg * kGK, g.group, &vfull[nA], pol);
+          tma_load_3d(dst + kGV / 2, &vmap, kGBox, sg * kGK, g.group, &vfull[nA], pol);
         }
       }
-      asm volatile("griddepcontrol.wait;" ::: "memory");  // the logits pass has completed
+      // (the logits are complete: see the weight warps)
       int t = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
@@ -647,7 +671,9 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
     const int quarter = warp & 3;
     const int dim = quarter * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // the brackets (and the logits) are complete
+    // No griddepcontrol.wait: this grid launches only after every bracket CTA
+    // has passed its own wait for the logits pass, so the logits, histograms
+    // and zeroed flags are complete; each row's bracket is waited for by flag.
     const float sc = p.scale2;
     int t = 0, jj = 0;
     bool ok = true;
@@ -660,6 +686,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
       float M = 0.0f;
       int llo = INT_MIN, lhi = INT_MAX;
       if (row_ok) {
+        if (!wait_bracket(tb.brk_ready + row)) ok = false;
         const RowBracket bk = ld_cg_bracket(tb.brk + row);
         M = bk.M;
         llo = bk.llo;
@@ -842,7 +869,7 @@ gather_tc_kernel(const __grid_constant__ CUtensorMap vmap, const float* __restri
 }
 
 template <int RT, bool ERR>
-cudaError_t launch_t(const CUtensorMap& map, const float* u, const unsigned char* vbase, const TcBufs& tb,
+cudaError_t launch_t(const CUtensorMap& map, const float* u, const TcBufs& tb,
                      float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   auto kern = gather_tc_kernel<RT, ERR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmem);
@@ -860,16 +887,16 @@ cudaError_t launch_t(const CUtensorMap& map, const float* u, const unsigned char
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, map, u, vbase, tb, acc, p, status);
+  return cudaLaunchKernelEx(&cfg, kern, map, u, tb, acc, p, status);
 }
 
 template <bool ERR>
-cudaError_t launch_e(const CUtensorMap& map, const float* u, const unsigned char* vbase, const TcBufs& tb,
+cudaError_t launch_e(const CUtensorMap& map, const float* u, const TcBufs& tb,
                      float* acc, const Plan& p, uint32_t* status, cudaStream_t st) {
   switch (p.rt_out) {
-    case 1: return launch_t<1, ERR>(map, u, vbase, tb, acc, p, status, st);
-    case 2: return launch_t<2, ERR>(map, u, vbase, tb, acc, p, status, st);
-    case 4: return launch_t<4, ERR>(map, u, vbase, tb, acc, p, status, st);
+    case 1: return launch_t<1, ERR>(map, u, tb, acc, p, status, st);
+    case 2: return launch_t<2, ERR>(map, u, tb, acc, p, status, st);
+    case 4: return launch_t<4, ERR>(map, u, tb, acc, p, status, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -984,7 +1011,8 @@ cudaError_t launch_bracket_tc(const float* cmax, const TcBufs& tb, const Plan& p
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, bracket_tc_kernel, (const RangeHist*)tb.hist, cmax, tb.brk, p);
+  return cudaLaunchKernelEx(&cfg, bracket_tc_kernel, (const RangeHist*)tb.hist, cmax, tb.brk,
+                            tb.brk_ready, p);
 }
 
 cudaError_t launch_gather_tc(const void* V, const float* u, const TcBufs& tb, float* acc,
@@ -992,9 +1020,8 @@ cudaError_t launch_gather_tc(const void* V, const float* u, const TcBufs& tb, fl
   if (p.rstages < 1) return cudaErrorInvalidValue;
   CUtensorMap map;
   if (!encode_kv_map(&map, V, p)) return cudaErrorInvalidValue;
-  const unsigned char* vb = static_cast<const unsigned char*>(V);
-  return p.want_err ? launch_e<true>(map, u, vb, tb, acc, p, status, st)
-                    : launch_e<false>(map, u, vb, tb, acc, p, status, st);
+  return p.want_err ? launch_e<true>(map, u, tb, acc, p, status, st)
+                    : launch_e<false>(map, u, tb, acc, p, status, st);
 }
 
 }  // namespace cta

@@ -149,6 +149,7 @@ score_kv_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16
        i += (int64_t)gridDim.x * kSThreads) {
     tb.cand_cnt[i] = 0u;
     tb.ticket[i] = 0u;
+    tb.brk_ready[i] = 0u;
   }
 
   if (warp == 0) {
