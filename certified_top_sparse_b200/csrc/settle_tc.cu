@@ -1027,8 +1027,17 @@ full_sort:
   {
     const int a = tid / kTD, dim = tid % kTD;
     double s = 0.0;
-    if (ERR || a == 0)
-      for (int c = 0; c < nr; ++c) s += (double)__ldcg(acc + ((row * nr + c) * 2 + a) * kTD + dim);
+    if (ERR || a == 0) {
+      // the ranges' partials in order, eight loads in flight
+      const float* src = acc + (row * nr * 2 + a) * kTD + dim;
+      for (int c0 = 0; c0 < nr; c0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = c0 + j < nr ? __ldcg(src + (int64_t)(c0 + j) * 2 * kTD) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s += (double)x[j];
+      }
+    }
     fin[a * kTD + dim] = s;
   }
   if (warp == 0) {  // the row's weight sums (for KL) and largest dropped logit, range order
