@@ -1,6 +1,6 @@
-// Phase 2-3 for decode-shaped problems (bf16 values, d = 128): the value pass
-// on the 5th-generation tensor cores, which needs only a bracket of the cut,
-// not the cut itself.
+// Kernels 2 and 3 of the decode path (bf16 values, d = 128): the row brackets
+// and the value pass on the 5th-generation tensor cores, which needs only a
+// bracket of the cut, not the cut itself.
 //
 // Method ("A Mathematical Theory of Top-k Sparse Attention via Total Variation
 // Distance", arXiv 2512.07647, abstract): certified Top-k keeps the minimal
@@ -10,7 +10,7 @@
 // sum_{kept} w_i v_i and the dropped sum sum_{dropped} w_i v_i.
 //
 // The bracket.  From the level histograms of the logits pass (RangeHist) the
-// weight warps bound, for every level boundary, the mass of the keys below it
+// bracket kernel bounds, for every level boundary, the mass of the keys below it
 // from above and from below (a level is 1/64 of a halving of the weight, so
 // every key's weight is known within a factor 2^(1/64) from its level alone),
 // and the total mass likewise.  The cut lies where the mass below reaches eps
@@ -48,12 +48,12 @@
 //   warp 1     MMA: 8 MMAs (K = 16) per stage, whose commit frees the slot; at
 //              the end of an item a commit hands the accumulator over; owns
 //              the tensor memory (two accumulators);
-//   warps 2-5  weights: warp r computes row r's bracket once per work item,
-//              then writes row r's part of each stage's W tile and its masses;
-//              at the end of an item the four warps read the accumulator
-//              (each its quarter of the tensor-memory lanes), add the parts in
-//              fp64 and write the range partials.  (Six warps: two per SM
-//              sub-partition at most, so the kernel may use 255 registers.)
+//   warps 2-9  weights: warp 2 + r + 4 h writes row r's part of the W tile
+//              and its masses in the stages of parity h (so two stages are in
+//              the works at once), after its row's bracket is out; at the end
+//              of an item the eight warps read the accumulator (each the
+//              tensor-memory lane quarter of its warp % 4), add the parts in
+//              fp64 and write the range partials.
 // Work items are (KV group, key range, row tile) with ranges cut in stages so
 // that every SM gets about the same number of stages.
 //
