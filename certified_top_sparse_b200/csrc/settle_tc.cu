@@ -62,11 +62,12 @@ constexpr int kSubMax = 512;             // sub-level bins of the cut search
 constexpr int kSubList = 256;            // keys of the cut's sub-level that are sorted
 constexpr int kWList = 256;              // per-warp list of window keys awaiting their value rows
 constexpr int kMaskBlock = 4 * kTThreads;  // mask words per block of the index writes (4 per thread)
-constexpr int kVPre = 128;
-constexpr int kStageWords = 124;         // mask words per staging round (124 x 32 + 3 <= 4096 slots)               // window value rows copied in while the cut is searched
+constexpr int kVPre = 128;               // window value rows copied in while the cut is searched
+constexpr int kStageWords = 124;         // mask words per staging round (124 x 32 + 3 <= 4096 slots)
 
-static_assert(kCandCap * 2 >= kStageWords * 32 + 3 && kVPre * kTD / 2 >= kStageWords * 32 + 3,
-              "the candidate list and the window rows double as the staging areas");
+static_assert(kCandCap * 2 >= kStageWords * 32 + 3 && kVPre * kTD / 2 >= 2 * kStageWords * 32 + 3 &&
+                  kTWarps * kWList * 2 >= kStageWords * 32 + 3,
+              "the candidate list, the window rows and the flat list double as the staging areas");
 
 struct SettleShared {
   alignas(16) unsigned long long cand[kCandCap];  // the row's candidates (sorted in place by the fallback)
@@ -119,6 +120,9 @@ __device__ __forceinline__ void bulk_wait_read() {
 }
 __device__ __forceinline__ void bulk_wait_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read2() {
+  asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -892,17 +896,26 @@ full_sort:
         // index i at slot i - g0 + pad so that a 16-byte boundary of idx_out is
         // one of the staging area; the aligned middle goes out as one bulk
         // copy, the (at most three) indices at either end as plain stores.
-        // Two staging areas take turns (the candidate list and the window
-        // rows, both read by now), so that a round's compaction overlaps the
-        // previous round's bulk copy.
+        // Staging areas take turns: the candidate list (kStageWords words)
+        // and the window rows (2 kStageWords), both read by now, and in the
+        // segment's last block of mask words also the flat window list
+        // (kStageWords), so that a round's compaction overlaps the earlier
+        // rounds' bulk copies and a segment of up to 16K keys needs no wait.
         const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(dst) >> 2) & 3u;
-        for (int s0 = 0, rnd = 0; s0 < nwb; s0 += kStageWords, ++rnd) {
-          int* stage = (rnd & 1) ? reinterpret_cast<int*>(&S.vrow[0][0]) : reinterpret_cast<int*>(S.cand);
-          if (rnd >= 2) {  // this area's copy of two rounds ago has read it
-            if (tid == 0) bulk_wait_read1();
+        const int nareas = (wb0 + kMaskBlock >= w_hi) ? 3 : 2;
+        for (int s0 = 0, rnd = 0; s0 < nwb; ++rnd) {
+          const int area = rnd % nareas;
+          int* stage = area == 0 ? reinterpret_cast<int*>(S.cand)
+                       : area == 1 ? reinterpret_cast<int*>(&S.vrow[0][0])
+                                   : reinterpret_cast<int*>(&S.wl_key[0][0]);
+          if (rnd >= nareas) {  // this area's copy of nareas rounds ago has read it
+            if (tid == 0) {
+              if (nareas == 3) bulk_wait_read2();
+              else bulk_wait_read1();
+            }
             __syncthreads();
           }
-          const int s1 = min(nwb, s0 + kStageWords);
+          const int s1 = min(nwb, s0 + (area == 1 ? 2 : 1) * kStageWords);
           const uint32_t off0 = S.u.mk.off[s0];
           const uint32_t off1 = s1 < nwb ? S.u.mk.off[s1] : S.off_win;
           // global positions [g0, g1) (never past n, whatever the records say)
@@ -938,6 +951,7 @@ full_sort:
             if (a1 > a0) bulk_store(dst + a0, stage + (a0 - g0 + pad), (a1 - a0) * 4u);
             bulk_commit();  // one group per round (possibly empty)
           }
+          s0 = s1;
         }
         if (tid == 0) bulk_wait_read();  // both areas may be written again
         __syncthreads();
