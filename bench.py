@@ -191,6 +191,21 @@ def algorithmic_bytes(prob, k_rows=None) -> dict:
             "idx_write": idx}
 
 
+def decode_config(workload: str, prob, eps: float, world: int) -> dict:
+    """The bench line's `config` for a decode workload (the same in both arms)."""
+    nq = len(prob.meta["q_steps"]) if "q_steps" in prob.meta else 1
+    kv = 2 * prob.batch * prob.n_kv_heads * prob.n * prob.d * prob.K.element_size()
+    return {
+        "workload": (f"{workload}: batch {prob.batch}, {prob.n_heads} query heads, "
+                     f"{prob.n_kv_heads} KV heads, d={prob.d}, n={prob.n}, bf16 KV cache "
+                     f"(sink/window/needle structure), eps={eps}, "
+                     + ("fresh queries each step (64-step cycle)" if nq > 1 else "fixed queries")),
+        "input_dtype": "bf16", "query_heads_per_step": prob.rows, "err_and_kl": True,
+        "l2": "inputs larger than L2 (K+V %.0f MB per step); no flush" % (kv / 1e6),
+        "parallelism": f"replicas x{world}",
+    }
+
+
 def run_libcta(args, rank, world, local_rank) -> dict | None:
     import torch
     import certified_top_sparse_b200 as cta
@@ -418,15 +433,7 @@ def run_libcta(args, rank, world, local_rank) -> dict | None:
         "warmup": args.warmup, "ms_per_step": seconds * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": (f"{args.workload}: batch {prob.batch}, {prob.n_heads} query heads, "
-                         f"{prob.n_kv_heads} KV heads, d={prob.d}, n={prob.n}, bf16 KV cache "
-                         f"(sink/window/needle structure), eps={eps}, "
-                         + ("fresh queries each step (64-step cycle)" if nq > 1 else "fixed queries")),
-            "input_dtype": "bf16", "query_heads_per_step": rows, "err_and_kl": True,
-            "l2": "inputs larger than L2 (K+V %.0f MB per step); no flush" % (nbytes["step"] / 1e6),
-            "parallelism": f"replicas x{world}",
-        },
+        "config": decode_config(args.workload, prob, eps, world),
         "roofline": {
             "bound": "hbm", "kernel": DECODE_KERNELS[dom_name], "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak if achieved else None,
@@ -733,7 +740,8 @@ def run_reference(args, rank, world) -> dict | None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload} (fp64 CPU oracle)", "eps": prob.eps},
+        "config": decode_config(args.workload, prob,
+                                args.eps if args.eps is not None else prob.eps, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
