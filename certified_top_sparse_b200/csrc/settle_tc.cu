@@ -1,4 +1,4 @@
-// Phase 4 of the tensor-core decode path (bf16 values, d = 128): the exact
+// Kernel 4 of the tensor-core decode path (bf16 values, d = 128): the exact
 // cut, the kept indices and the outputs of every row.
 //
 // Method ("A Mathematical Theory of Top-k Sparse Attention via Total Variation
@@ -10,32 +10,34 @@
 //
 // The value pass has already summed the values and exact masses of the keys
 // whose side of the cut its bracket decided (kept: level >= lhi; dropped:
-// level < llo); what is left is the window between.  One CTA per (row, key
-// range) - the ranges of the value pass - so the row's work spreads over
-// nranges CTAs:
-//   1. Row totals from the range records: Z, the dropped mass D below the
-//      window, the window mass W and the kept count.  The bracket is checked
-//      exactly: D / Z <= eps < (D + W) / Z must hold, i.e. the cut lies in
-//      the window.  (If it did not - which the value pass's rigorous bounds
-//      exclude - the row is recomputed here from the logits alone, with every
-//      key treated as a window key, and CTA_DEV_INTERNAL is set.)
-//   2. The exact cut.  Usually all the window's keys are in the row's
-//      candidate list (composite keys: logit order, then index).  Every CTA
-//      of the row sums their exact 2^-62 masses per sub-level (1/4096 of a
-//      halving of the weight, an interval of the ranking), finds the sub-level
-//      where the certificate starts to hold, sorts only that sub-level's keys
-//      and walks them to the last kept key.  Otherwise (a window wider than
-//      the sub-level table, or more window keys than the list holds, e.g. many
-//      tied logits) a full sort of the list, or a radix select over the 64-bit
-//      composite keys of the window, eight bits per pass over the row's
-//      logits, with exact 128-bit digit masses.
-//   3. The CTA's key range: its kept indices, ascending, at the offset of the
-//      kept keys before it (kept counts of the ranges before + window keys
-//      kept before it), from the logits with all loads of a batch in flight
-//      and one block scan per batch; and the value rows of its window keys,
-//      gathered (256-byte rows, eight in flight per warp) and added to the
-//      kept or dropped side, on top of the value pass's range partial, with
-//      the weight sums for KL and the largest dropped logit.
+// level < llo), marked the kept-for-certain keys in a bit mask and listed the
+// keys between (the window) as candidates.  One CTA per (row, segment of
+// Plan::settle_group value-pass ranges):
+//   1. Inputs: the row's candidate list and the segment's mask words come in
+//      by bulk copies (one mbarrier); row totals from the range records: Z,
+//      the dropped mass D below the window, the window mass W and the kept
+//      count.  The bracket is checked exactly: D / Z <= eps < (D + W) / Z must
+//      hold, i.e. the cut lies in the window.  (If it did not - which the
+//      bracket's rigorous bounds exclude - the row is recomputed here from the
+//      logits alone, with every key treated as a window key, and
+//      CTA_DEV_INTERNAL is set.)
+//   2. The exact cut.  Usually all the window's keys are in the candidate
+//      list (composite keys: logit order, then index).  Every CTA of the row
+//      sums their exact 2^-62 masses per sub-level (1/4096 of a halving of the
+//      weight, an interval of the ranking), finds the sub-level where the
+//      certificate starts to hold, sorts only that sub-level's keys and walks
+//      them to the last kept key.  Otherwise (cold paths, out of line: a
+//      window wider than the sub-level table, more window keys than the list
+//      holds, e.g. many tied logits) a full sort of the list, or a radix
+//      select over the 64-bit composite keys of the window, eight bits per
+//      pass over the row's logits, with exact 128-bit digit masses.
+//   3. The segment: its window keys' value rows (bulk copies, issued before
+//      the cut search) added to the kept or dropped side, with the weight sums
+//      for KL and the largest dropped logit; its kept indices, ascending, at
+//      the offset of the kept keys before it: the mask words OR the kept
+//      window keys, compacted in shared memory and written by bulk stores
+//      (staging areas taking turns).  Without a usable candidate list the
+//      segment's logits are scanned instead (cold path).
 //   4. The last CTA of the row (a ticket counter that the logits pass zeroes)
 //      adds the range partials in a fixed order and writes out, err, KL, k,
 //      TV and the single-gap bound.  The output normalisers are the exact
