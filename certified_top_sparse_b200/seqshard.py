@@ -60,11 +60,11 @@ def _all_gather_padded(t: torch.Tensor, group) -> list[torch.Tensor]:
     if not (dist.is_available() and dist.is_initialized()):
         return [t]
     world = dist.get_world_size(group)
-    cnt = torch.tensor([t.shape[0]], dtype=torch.int64)
+    cnt = torch.tensor([t.shape[0]], dtype=torch.int64, device=t.device)
     cnts = [torch.zeros_like(cnt) for _ in range(world)]
     dist.all_gather(cnts, cnt, group=group)
     mx = int(max(c.item() for c in cnts))
-    pad = torch.zeros((mx, *t.shape[1:]), dtype=t.dtype)
+    pad = torch.zeros((mx, *t.shape[1:]), dtype=t.dtype, device=t.device)
     pad[: t.shape[0]] = t
     outs = [torch.zeros_like(pad) for _ in range(world)]
     dist.all_gather(outs, pad, group=group)
@@ -131,47 +131,49 @@ def certify_sharded(s: torch.Tensor, V: torch.Tensor, key0: int, eps: float, gro
     """
     import torch.distributed as dist
     rows, nl = s.shape
+    dev = s.device  # every exchanged tensor lives here (a GPU for NCCL, the CPU for gloo)
     s = s.to(torch.float64)
-    V = V.to(torch.float64)
+    V = V.to(device=dev, dtype=torch.float64)
     # 1. the row maxima
-    M = s.max(dim=1).values if nl else torch.full((rows,), -math.inf, dtype=torch.float64)
+    M = s.max(dim=1).values if nl else torch.full((rows,), -math.inf, dtype=torch.float64, device=dev)
     _all_reduce(M, dist.ReduceOp.MAX, group)
     a = (M[:, None] - s) * (1.0 / math.log(2.0))           # log2(w_max / w) >= 0
     w = torch.exp2(-a)
     # 2. level counts in the common frame
     G = LEVELS * FRAME_OCTAVES
     gi = torch.floor(a * LEVELS).to(torch.int64)
-    counts = torch.zeros((rows, G), dtype=torch.int64)
+    counts = torch.zeros((rows, G), dtype=torch.int64, device=dev)
     inframe = gi < G
     counts.scatter_add_(1, torch.where(inframe, gi, 0), inframe.to(torch.int64))
     deep = (~inframe).sum(dim=1)
     _all_reduce(counts, dist.ReduceOp.SUM, group)
     _all_reduce(deep, dist.ReduceOp.SUM, group)
-    g_lo, g_hi = bracket(counts, deep, eps)
-    glo = torch.tensor(g_lo, dtype=torch.int64)[:, None]
-    ghi = torch.tensor(g_hi, dtype=torch.int64)[:, None]
+    g_lo, g_hi = bracket(counts.cpu(), deep.cpu(), eps)
+    glo = torch.tensor(g_lo, dtype=torch.int64, device=dev)[:, None]
+    ghi = torch.tensor(g_hi, dtype=torch.int64, device=dev)[:, None]
     head = gi < ghi
     tail = gi >= glo
     win = ~head & ~tail
     # 3. exact masses above, inside and below the bracket
-    m = torch.round(torch.ldexp(w, torch.tensor(MASS_BITS))).to(torch.int64)
+    m = torch.round(torch.ldexp(w, torch.tensor(MASS_BITS, device=dev))).to(torch.int64)
     sums = torch.stack([_limbs(torch.where(head, m, 0)), _limbs(torch.where(win, m, 0)),
                         _limbs(torch.where(tail, m, 0))], dim=1)  # [rows, 3, 2]
     _all_reduce(sums, dist.ReduceOp.SUM, group)
+    sums_h = sums.cpu()
     # 4. the window keys, gathered; the exact cut
-    gidx = torch.arange(key0, key0 + nl, dtype=torch.int64)
+    gidx = torch.arange(key0, key0 + nl, dtype=torch.int64, device=dev)
     cuts = []
     for r in range(rows):
         sel = torch.nonzero(win[r]).flatten()
-        mine = torch.stack([s[r, sel], gidx[sel].to(torch.float64), m[r, sel].to(torch.float64)], 1) \
-            if len(sel) else torch.zeros((0, 3), dtype=torch.float64)
-        # masses travel as exact integers: split into two exact fp64 halves
+        mine = torch.stack([s[r, sel], gidx[sel].to(torch.float64)], 1) \
+            if len(sel) else torch.zeros((0, 2), dtype=torch.float64, device=dev)
+        # masses travel as exact integers, in two 31-bit halves
         mine_m = torch.stack([m[r, sel] >> LIMB, m[r, sel] & ((1 << LIMB) - 1)], 1) \
-            if len(sel) else torch.zeros((0, 2), dtype=torch.int64)
-        allc = torch.cat(_all_gather_padded(mine, group), 0)
-        allm = torch.cat(_all_gather_padded(mine_m, group), 0)
-        Zr = sum(_from_limbs(sums[r, j]) for j in range(3))
-        C = _from_limbs(sums[r, 0])
+            if len(sel) else torch.zeros((0, 2), dtype=torch.int64, device=dev)
+        allc = torch.cat(_all_gather_padded(mine, group), 0).cpu()
+        allm = torch.cat(_all_gather_padded(mine_m, group), 0).cpu()
+        Zr = sum(_from_limbs(sums_h[r, j]) for j in range(3))
+        C = _from_limbs(sums_h[r, 0])
         # ranking: logit descending, then index ascending
         order = sorted(range(allc.shape[0]), key=lambda i: (-float(allc[i, 0]), int(allc[i, 1])))
         cut = None
@@ -196,13 +198,14 @@ def certify_sharded(s: torch.Tensor, V: torch.Tensor, key0: int, eps: float, gro
     _all_reduce(wsum, dist.ReduceOp.SUM, group)
     _all_reduce(nk, dist.ReduceOp.SUM, group)
     # 6. the kept indices, ascending over the ranks
-    idx = [torch.cat(_all_gather_padded(gidx[kept[r]], group), 0) for r in range(rows)]
+    idx = [torch.cat(_all_gather_padded(gidx[kept[r]], group), 0).cpu() for r in range(rows)]
+    part, wsum, nk = part.cpu(), wsum.cpu(), nk.cpu()
     out = torch.zeros((rows, V.shape[-1]), dtype=torch.float64)
     tv = torch.zeros(rows, dtype=torch.float64)
     kl = torch.zeros(rows, dtype=torch.float64)
     err = torch.zeros(rows, dtype=torch.float64)
     for r in range(rows):
-        Zr = sum(_from_limbs(sums[r, j]) for j in range(3))
+        Zr = sum(_from_limbs(sums_h[r, j]) for j in range(3))
         C = cuts[r][2]
         tv[r] = float(Z_minus := Zr - C) / float(Zr)
         hm = math.ldexp(float(C), -MASS_BITS)
