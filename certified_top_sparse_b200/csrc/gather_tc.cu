@@ -139,6 +139,8 @@ __device__ __forceinline__ bool wait_bracket(const uint32_t* ready) {
       }
     }
   }
+  // the warp barrier orders lane 0's acquire before every lane's reads of the bracket
+  __syncwarp();
   return __shfl_sync(0xffffffffu, ok, 0) != 0u;
 }
 
