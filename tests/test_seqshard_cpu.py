@@ -40,18 +40,31 @@ def shard_inputs(q, K, V, lo, hi):
     return s, torch.from_numpy(V[0, :, lo:hi, :]).double()
 
 
+def tied_problem():
+    """Logits on a coarse grid (many exact ties, also across the shard
+    boundary): the cut falls inside a run of equal logits, so the lower index
+    must win across ranks."""
+    rng = np.random.default_rng(777)
+    q = np.zeros((1, ROWS, 1, D), np.float32)
+    q[..., 0] = 1.0
+    K = np.zeros((1, ROWS, N, D), np.float32)
+    K[..., 0] = (rng.integers(0, 6, size=(1, ROWS, N)) * 2.0).astype(np.float32)  # logits 0, .25, ... 1.25
+    V = rng.standard_normal((1, ROWS, N, D)).astype(np.float32)
+    return q, K, V
+
+
 WORKER = r"""
 import json, os, sys
 sys.path.insert(0, %(root)r)
 sys.path.insert(0, os.path.join(%(root)r, "tests"))
 import torch
 import torch.distributed as dist
-from test_seqshard_cpu import problem, shard_inputs, N, EPS
+from test_seqshard_cpu import problem, tied_problem, shard_inputs, N, EPS
 from certified_top_sparse_b200 import seqshard
 import datetime
 dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
 rank, world = dist.get_rank(), dist.get_world_size()
-q, K, V = problem()
+q, K, V = tied_problem() if os.environ.get("CTA_TIED") else problem()
 bounds = [0, 2999, N]          # an odd split
 s, v = shard_inputs(q, K, V, bounds[rank], bounds[rank + 1])
 r = seqshard.certify_sharded(s, v, bounds[rank], EPS)
@@ -82,8 +95,8 @@ def _check(res, ora):
     assert np.all(np.abs(out - ora["out"]) <= 1e-10 * scale)
 
 
-def _oracle():
-    q, K, V = problem()
+def _oracle(make=problem):
+    q, K, V = make()
     return oracle.certified_topk_attn(q, K, V, EPS, n_heads=ROWS, n_kv_heads=ROWS, dtype=oracle.F32)
 
 
@@ -95,7 +108,8 @@ def test_one_process_matches_oracle():
             "err": r["err"].numpy(), "out": r["out"].numpy()}, _oracle())
 
 
-def test_two_gloo_ranks_match_oracle(tmp_path):
+@pytest.mark.parametrize("tied", [False, True])
+def test_two_gloo_ranks_match_oracle(tmp_path, tied):
     script = tmp_path / "worker.py"
     script.write_text(WORKER % {"root": ROOT})
     port = _free_port()
@@ -103,6 +117,8 @@ def test_two_gloo_ranks_match_oracle(tmp_path):
     for rank in range(2):
         env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
                    MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        if tied:
+            env["CTA_TIED"] = "1"
         procs.append(subprocess.Popen([sys.executable, str(script)], env=env,
                                       stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
     outs = []
@@ -110,7 +126,7 @@ def test_two_gloo_ranks_match_oracle(tmp_path):
         o, e = p.communicate(timeout=180)
         assert p.returncode == 0, e
         outs.append(json.loads(o.strip().splitlines()[-1]))
-    ora = _oracle()
+    ora = _oracle(tied_problem if tied else problem)
     for res in outs:  # every rank holds the whole result
         _check(res, ora)
     assert outs[0]["idx"] == outs[1]["idx"] and outs[0]["out"] == outs[1]["out"]
