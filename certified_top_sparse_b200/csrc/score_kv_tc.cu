@@ -41,9 +41,9 @@
 // the stream (the caller's, or the previous call's last kernel).  Every
 // thread waits for that grid (griddepcontrol.wait) before anything reads q or
 // K or writes the workspace; only the tensor-memory allocation, the barrier
-// set-up and the tensor-map prefetch come first.  It then lets the value pass
-// launch (it can only start on an SM once this kernel's CTA there has left)
-// and zeroes the per-row counters that the value pass and the last kernel use.
+// set-up and the tensor-map prefetch come first.  It then lets the bracket
+// kernel launch and zeroes the per-row counters and flags that the later
+// kernels of the call use.
 #include <algorithm>
 
 #include "common.cuh"
