@@ -143,3 +143,32 @@ def test_bracket_contains_the_cut_on_a_two_level_row():
     need = int(np.ceil(1000 - 0.05 * Z * 2 ** 12))
     assert int(r["k"][0]) == 10 + max(0, need)
     assert r["tv"][0] <= 0.05
+
+
+@pytest.mark.parametrize("seed,sigma,eps", [(1, 1.0, 0.01), (2, 3.0, 0.001), (3, 0.3, 0.1),
+                                            (4, 6.0, 1e-4), (5, 1.5, 0.5)])
+def test_bracket_brackets_the_oracles_cut(seed, sigma, eps):
+    # From the level counts alone, every key below bin g_hi must be one the
+    # oracle keeps and every key from bin g_lo on one it drops.
+    rng = np.random.default_rng(seed)
+    n = 20000
+    s = rng.standard_normal(n) * sigma
+    s[rng.integers(0, n, 5)] += 4 * sigma  # a few large logits
+    s = s.astype(np.float32)               # the oracle's inputs: q = 1, d = 1, K = s
+    ora = oracle.certified_topk_attn(np.ones((1, 1, 1, 1), np.float32), s.reshape(1, 1, n, 1),
+                                     np.zeros((1, 1, n, 1), np.float32), eps,
+                                     n_heads=1, n_kv_heads=1, dtype=oracle.F32)
+    kept = np.zeros(n, bool)
+    kept[ora["idx"][0]] = True
+    assert kept.sum() == ora["k"][0]
+    s64 = s.astype(np.float64)
+    a = (s64.max() - s64) / np.log(2.0)
+    g = np.floor(a * seqshard.LEVELS).astype(np.int64)
+    G = seqshard.LEVELS * seqshard.FRAME_OCTAVES
+    counts = np.bincount(g[g < G], minlength=G)[None, :]
+    deep = np.array([(g >= G).sum()])
+    g_lo, g_hi = seqshard.bracket(torch.from_numpy(counts), torch.from_numpy(deep), eps)
+    g_lo, g_hi = g_lo[0], g_hi[0]
+    assert g_hi < g_lo
+    assert kept[g < g_hi].all()
+    assert not kept[g >= g_lo].any()
